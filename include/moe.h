@@ -1,0 +1,213 @@
+/*
+ * moe.h -- C ABI of libmoe: the DeepSeekMoE layer forward on NVIDIA B200
+ * (sm_100a).
+ *
+ * The layer (from "DeepSeekMoE: Towards Ultimate Expert Specialization in
+ * Mixture-of-Experts Language Models", §3.2 Shared Expert Isolation,
+ * eqs. (9)-(11)):
+ *
+ *   h_t  = u_t + sum_{s < K_s} FFN_s(u_t) + sum_{k < K} g_{t,k} FFN_{idx[t,k]}(u_t)
+ *   s_t  = Softmax_i(u_t^T e_i (+ b_i))   over the N_r routed experts
+ *   idx  = the K largest s_{t,i} (lower expert index wins ties),
+ *   g    = s at those experts, not renormalised
+ *   FFN(x) = W2 (SiLU(W1 x) * (W3 x))    (SwiGLU, no biases)
+ *
+ * with N_r = mN - K_s fine-grained routed experts (§3.1) and K = mK - K_s.
+ * Layer normalisation is not part of the layer (the pages omit it, §2).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers are DEVICE pointers owned by the caller unless a parameter says
+ *   HOST.  The library never allocates device memory; scratch space comes
+ *   from the caller's workspace `ws` (size from moe_workspace_size).
+ * - All tensors are dense row-major.  Element types: `dtype` MOE_DTYPE_BF16
+ *   means activations and weights are bfloat16 (raw 16-bit); MOE_DTYPE_F32
+ *   means float32.  Router bias, gates and fp32 intermediates are float32;
+ *   indices are int32.
+ * - Base pointers must be 16-byte aligned (MOE_ERR_ALIGN otherwise).
+ * - The bf16 path runs the expert GEMMs on tcgen05 tensor cores and needs
+ *   d % 64 == 0 and inter % 64 == 0; the fp32 path runs them on CUDA cores.
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *   default stream) and never synchronises the host, except where stated.
+ * - Return value: MOE_OK (0) or a negative MOE_ERR_* code.  Nothing is
+ *   launched after a validation error.  MOE_ERR_CUDA reports a launch error.
+ *   A kernel that gives up on a bounded wait records MOE_ERR_DEVICE_CHECK in
+ *   the workspace's status word, read with moe_read_status.
+ * - Results are bitwise reproducible from run to run (no atomics decide any
+ *   value or order).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* moe_stream_t; /* a cudaStream_t */
+
+enum {
+  MOE_DTYPE_F32 = 0,
+  MOE_DTYPE_BF16 = 1,
+};
+
+enum {
+  MOE_OK = 0,
+  MOE_ERR_NULLPTR = -1,      /* a required pointer is NULL */
+  MOE_ERR_SHAPE = -2,        /* sizes out of range or inconsistent */
+  MOE_ERR_ALIGN = -3,        /* a pointer is not 16-byte aligned */
+  MOE_ERR_WORKSPACE = -4,    /* workspace smaller than moe_workspace_size */
+  MOE_ERR_DTYPE = -5,        /* unknown dtype */
+  MOE_ERR_CUDA = -6,         /* CUDA runtime / launch error */
+  MOE_ERR_DEVICE_CHECK = -7, /* a kernel gave up waiting (see moe_read_status) */
+  MOE_ERR_UNSUPPORTED = -8,  /* no device of compute capability 10.0 */
+};
+
+/* Router flags (moe_shape_t.flags). */
+enum {
+  /* The router bias b_i shifts only the top-K selection; the gates are the
+     softmax of the unbiased logits (the per-expert load-balancing bias the
+     csdn.net DeepSeekMoE article describes in words, §2.3).  Default (0):
+     the bias is part of the logit for both selection and softmax. */
+  MOE_FLAG_BIAS_SELECT_ONLY = 1,
+};
+
+/* Layer shape.  Limits: 1 <= n_routed <= 256, 1 <= top_k <= min(n_routed, 32),
+   0 <= n_shared <= 64, T >= 0 (T = 0 is a no-op), d >= 1, inter >= 1.  */
+typedef struct {
+  int64_t T;        /* tokens */
+  int32_t d;        /* hidden size */
+  int32_t n_routed; /* N_r = mN - K_s routed experts */
+  int32_t n_shared; /* K_s shared experts */
+  int32_t inter;    /* I, intermediate width of one fine-grained expert */
+  int32_t top_k;    /* K = mK - K_s routed experts per token */
+  int32_t dtype;    /* MOE_DTYPE_* */
+  int32_t flags;    /* MOE_FLAG_* */
+} moe_shape_t;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_strerror(int status);
+
+/* Bytes of workspace that moe_layer_forward, moe_dispatch and
+   moe_expert_ffn need for `shape` (a multiple of 256). */
+int moe_workspace_size(const moe_shape_t* shape, size_t* bytes);
+
+/* W13 packing used by the tensor-core gate/up GEMM.
+   W1, W3: [n_experts, inter, d]; W13 out: [n_experts, 2*inter, d] where, for
+   every block b of 64 intermediate rows, packed rows 128b..128b+63 are W1
+   rows 64b..64b+63 and packed rows 128b+64..128b+127 are W3 rows 64b..64b+63.
+   (For dtype F32 the packed layout is the same.)  inter % 64 must be 0.
+   Weight preparation, done once per model, not per forward. */
+int moe_pack_w13(const moe_shape_t* shape, int32_t n_experts, const void* W1,
+                 const void* W3, void* W13, moe_stream_t stream);
+
+/* a1-a2, router (eqs. (10)-(11)): logits u_t.e_i (+ b_i) accumulated in fp32
+   in order j = 0..d-1, softmax over the n_routed experts, top-K.
+   u: [T, d]; E: [n_routed, d]; bias: [n_routed] float32 or NULL.
+   Outputs idx: [T, top_k] int32 in descending score order (ties: lower
+   index first); w: [T, top_k] float32 gates (not renormalised). */
+int moe_route(const moe_shape_t* shape, const void* u, const void* E,
+              const float* bias, int32_t* idx, float* w, moe_stream_t stream);
+
+/* a3, dispatch ("each token is computed only by its K experts", §2):
+   counts[e] = #{(t,k): idx[t,k] = e}; offsets = exclusive scan (n_routed+1);
+   perm[p] = slot t*top_k+k of position p, expert e's slots filling
+   offsets[e]..offsets[e+1]-1 in increasing t; inv[t*top_k+k] = its position.
+   idx must hold distinct experts per token in [0, n_routed).
+   All outputs int32; bit-exact.  Uses workspace `ws`. */
+int moe_dispatch(const moe_shape_t* shape, const int32_t* idx, int32_t* counts,
+                 int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
+                 size_t ws_bytes, moe_stream_t stream);
+
+/* a4-a6, expert FFNs: for every position p of expert e's segment,
+   y[p] = FFN_e(u_{perm[p]/top_k}); and ysh[t] = sum_s FFN_s(u_t) over the
+   shared experts (computed as one SwiGLU FFN of width n_shared*inter, the
+   segmentation identity of §3.1).
+   W13: [n_routed, 2*inter, d] packed by moe_pack_w13; W2: [n_routed, d, inter];
+   W13_s: [n_shared, 2*inter, d] packed; W2_s: [n_shared, d, inter].
+   y: [T*top_k, d] in dtype; ysh: [T, d] float32.  fp32 accumulation; for bf16
+   the SwiGLU activation is rounded to bf16 before the down projection.
+   perm/offsets as produced by moe_dispatch.  Uses workspace `ws`. */
+int moe_expert_ffn(const moe_shape_t* shape, const void* u, const int32_t* perm,
+                   const int32_t* offsets, const void* W13, const void* W2,
+                   const void* W13_s, const void* W2_s, void* y, float* ysh,
+                   void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* a7, combine + residual (eq. (9)): h_t = u_t + ysh_t + sum_{k<K} w[t,k] *
+   y[inv[t*K+k]], accumulated in fp32 in exactly that order, rounded once to
+   dtype.  h: [T, d] dtype. */
+int moe_combine(const moe_shape_t* shape, const void* u, const float* ysh,
+                const void* y, const float* w, const int32_t* inv, void* h,
+                moe_stream_t stream);
+
+/* The whole layer: route, dispatch, expert FFNs and combine, on `stream`,
+   with every intermediate in `ws`.  Arguments as above; h: [T, d] dtype. */
+int moe_layer_forward(const moe_shape_t* shape, const void* u, const void* E,
+                      const float* bias, const void* W13, const void* W2,
+                      const void* W13_s, const void* W2_s, void* h, void* ws,
+                      size_t ws_bytes, moe_stream_t stream);
+
+/* moe_layer_forward with the activations in HOST memory: u_host [T, d] is
+   copied to the device, the layer runs, and h is copied back into h_host, all
+   enqueued on `stream`; the call then waits for the stream.  Page-locked
+   host buffers make the copies asynchronous DMA.  Weights stay on the
+   device.  Workspace: moe_workspace_size plus 2*T*d*elem bytes. */
+int moe_layer_forward_host(const moe_shape_t* shape, const void* u_host,
+                           const void* E, const float* bias, const void* W13,
+                           const void* W2, const void* W13_s, const void* W2_s,
+                           void* h_host, void* ws, size_t ws_bytes,
+                           moe_stream_t stream);
+
+/* Bytes moe_layer_forward_host needs. */
+int moe_workspace_size_host(const moe_shape_t* shape, size_t* bytes);
+
+/* Expert load statistics of §3.3, eqs. (12)-(14), for the routing in idx
+   and the scores of the router: f[e] = N'/(K'T) * counts[e] and P[e] =
+   (1/T) sum_t s_{t,e}, with s recomputed from u, E, bias as in moe_route.
+   f, P: [n_routed] float32.  (Training statistic; not on the forward path.)
+   Uses workspace `ws`. */
+int moe_expert_balance(const moe_shape_t* shape, const void* u, const void* E,
+                       const float* bias, const int32_t* counts, float* f,
+                       float* P, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Copies the workspace status word (0 or MOE_ERR_DEVICE_CHECK) to *status
+   and clears it; synchronises `stream`. */
+int moe_read_status(const void* ws, int32_t* status, moe_stream_t stream);
+
+/* Tracing: device time of each stage.  While enabled, every kernel (the
+   three dispatch kernels count as one stage) that libmoe launches is
+   bracketed by CUDA events recorded on its stream.  moe_profile_read waits
+   for those events and returns, oldest first, the stage kind (MOE_KERNEL_*)
+   and elapsed milliseconds of each bracketed launch since the last read:
+   at most `max` entries are written and *count receives the number
+   written; up to 4096 are kept, later ones are dropped.  Enabling adds event
+   records between launches and never changes any result. */
+enum {
+  MOE_KERNEL_ROUTER = 1,
+  MOE_KERNEL_DISPATCH = 2,
+  MOE_KERNEL_GATHER = 3,
+  MOE_KERNEL_GEMM_GATE_UP = 4, /* grouped gate/up GEMM + SwiGLU (tcgen05) */
+  MOE_KERNEL_GEMM_DOWN = 5,    /* grouped down GEMM (tcgen05) */
+  MOE_KERNEL_COMBINE = 6,
+  MOE_KERNEL_FFN_F32 = 7,      /* the fp32 expert FFN (both GEMMs) */
+  MOE_KERNEL_MEMSET = 8,
+  MOE_KERNEL_PACK = 9,
+  MOE_KERNEL_BALANCE = 10,
+};
+int moe_profile_enable(int on);
+int moe_profile_read(int32_t* kinds, float* ms, int32_t max, int32_t* count);
+const char* moe_kernel_name(int32_t kind);
+
+/* Number of kernels this library has launched since load (all threads). */
+uint64_t moe_launch_count(void);
+
+/* Library version string. */
+const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

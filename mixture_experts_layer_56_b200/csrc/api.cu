@@ -1,0 +1,567 @@
+// C ABI of libmoe (include/moe.h): validation, workspace carving and the
+// launch sequence of the DeepSeekMoE layer forward on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "gemm_sm100.h"
+#include "kernels.h"
+
+namespace moe {
+
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+int check_launch() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// ---------------------------------------------------------------------------
+// tracing: CUDA events around each stage, on the stage's stream
+// ---------------------------------------------------------------------------
+namespace {
+struct ProfRec {
+  int32_t kind;
+  cudaEvent_t beg, end;
+};
+struct Profiler {
+  std::mutex mu;
+  std::atomic<bool> on{false};
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+};
+Profiler& prof() {
+  static Profiler p;
+  return p;
+}
+constexpr size_t kMaxProfRecs = 4096;
+
+// RAII bracket: records the start event now and the end event when it goes
+// out of scope (after the stage's launches were enqueued).
+class Stage {
+ public:
+  Stage(int32_t kind, cudaStream_t st) : st_(st) {
+    Profiler& p = prof();
+    if (!p.on.load()) return;
+    std::lock_guard<std::mutex> lock(p.mu);
+    if (p.recs.size() >= kMaxProfRecs) return;
+    ProfRec r{kind, p.get(), p.get()};
+    if (!r.beg || !r.end) return;
+    cudaEventRecord(r.beg, st_);
+    p.recs.push_back(r);
+    idx_ = static_cast<long>(p.recs.size()) - 1;
+  }
+  ~Stage() {
+    if (idx_ < 0) return;
+    Profiler& p = prof();
+    std::lock_guard<std::mutex> lock(p.mu);
+    cudaEventRecord(p.recs[static_cast<size_t>(idx_)].end, st_);
+  }
+
+ private:
+  cudaStream_t st_;
+  long idx_ = -1;
+};
+}  // namespace
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t round_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+struct Layout {
+  size_t status, idx, w, counts, offsets, perm, inv, chunk_counts, chunk_base, pstat;
+  size_t xperm, act, act_s, y, ysh, total;
+  size_t u_host, h_host, total_host;  // extra staging for moe_layer_forward_host
+};
+
+size_t elem_bytes(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+
+Layout layout_of(const moe_shape_t& s) {
+  const size_t T = static_cast<size_t>(s.T), K = s.top_k, n = s.n_routed, d = s.d,
+               I = s.inter, ns = s.n_shared, el = elem_bytes(s.dtype);
+  const size_t nch = static_cast<size_t>(dispatch_num_chunks(s.T));
+  const size_t nrc = static_cast<size_t>(router_num_ctas(s.T));
+  Layout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += round_up(bytes);
+    return at;
+  };
+  L.status = take(kAlign);
+  L.idx = take(T * K * 4);
+  L.w = take(T * K * 4);
+  L.counts = take(n * 4);
+  L.offsets = take((n + 1) * 4);
+  L.perm = take(T * K * 4);
+  L.inv = take(T * K * 4);
+  L.chunk_counts = take(nch * n * 4);
+  L.chunk_base = take(nch * n * 4);
+  L.pstat = take(nrc * n * 4);
+  L.xperm = take(T * K * d * el);
+  L.act = take(T * K * I * el);
+  L.act_s = take(T * ns * I * el);
+  L.y = take(T * K * d * el);
+  L.ysh = take(T * d * 4);
+  L.total = o;
+  L.u_host = take(T * d * el);
+  L.h_host = take(T * d * el);
+  L.total_host = o;
+  return L;
+}
+
+int validate(const moe_shape_t* s) {
+  if (!s) return MOE_ERR_NULLPTR;
+  if (s->dtype != MOE_DTYPE_F32 && s->dtype != MOE_DTYPE_BF16) return MOE_ERR_DTYPE;
+  if (s->T < 0 || s->d < 1 || s->n_routed < 1 || s->n_routed > 256 || s->top_k < 1 ||
+      s->top_k > s->n_routed || s->top_k > 32 || s->n_shared < 0 || s->n_shared > 64 ||
+      s->inter < 1)
+    return MOE_ERR_SHAPE;
+  if ((s->flags & ~MOE_FLAG_BIAS_SELECT_ONLY) != 0) return MOE_ERR_SHAPE;
+  // positions are int32; rows address TMA coordinates (int32)
+  if (s->T * static_cast<int64_t>(s->top_k) > 0x7fffffffLL) return MOE_ERR_SHAPE;
+  if (s->inter % 64 != 0) return MOE_ERR_SHAPE;
+  if (s->dtype == MOE_DTYPE_BF16) {
+    if (s->d % 64 != 0) return MOE_ERR_SHAPE;
+  } else {
+    if (s->d % 4 != 0) return MOE_ERR_SHAPE;
+  }
+  return MOE_OK;
+}
+
+inline bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+struct DeviceInfo {
+  int ok = -1;  // -1 unknown, 0 unsupported, 1 sm_100
+  int sms = 0;
+};
+
+int device_info(DeviceInfo* out) {
+  static DeviceInfo cache[64];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceInfo& di = cache[dev];
+  if (di.ok < 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    di.ok = (major == 10 && minor == 0) ? 1 : 0;
+    di.sms = sms;
+  }
+  *out = di;
+  return di.ok == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// expert FFNs on workspace-resident gathered rows
+int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const int32_t* perm,
+                   const int32_t* offsets, const void* W13, const void* W2, const void* W13_s,
+                   const void* W2_s, void* y, float* ysh, void* ws, cudaStream_t st, int sms) {
+  const int64_t T = s.T, K = s.top_k, rows = T * K;
+  const int d = s.d, I = s.inter, n = s.n_routed, ns = s.n_shared;
+  void* xperm = at<void>(ws, L.xperm);
+  void* act = at<void>(ws, L.act);
+  void* act_s = at<void>(ws, L.act_s);
+  {
+    Stage sg(MOE_KERNEL_GATHER, st);
+    if (int rc = launch_gather(s.dtype, u, perm, rows, d, static_cast<int>(K), xperm, st))
+      return rc;
+  }
+  if (ns == 0) {
+    // no shared experts: ysh = 0
+    Stage sg(MOE_KERNEL_MEMSET, st);
+    if (int rc = launch_zero(ysh, static_cast<size_t>(T) * d * 4, st)) return rc;
+  }
+
+  if (s.dtype == MOE_DTYPE_F32) {
+    const int max_mt = static_cast<int>((rows + 63) / 64 + (rows < n ? rows : n));
+    Stage sg(MOE_KERNEL_FFN_F32, st);
+    return launch_ffn_f32(static_cast<const float*>(xperm), static_cast<const float*>(u), offsets,
+                          n, T, ns, d, I, static_cast<const float*>(W13),
+                          static_cast<const float*>(W2), static_cast<const float*>(W13_s),
+                          static_cast<const float*>(W2_s), static_cast<float*>(act),
+                          static_cast<float*>(act_s), static_cast<float*>(y), ysh, max_mt, st);
+  }
+
+  using namespace sm100;
+  const uint64_t d64 = static_cast<uint64_t>(d), I64 = static_cast<uint64_t>(I);
+  const int64_t routed_mt_ub = (rows + 127) / 128 + (rows < n ? rows : n);
+  const int64_t shared_mt = ns > 0 ? (T + 127) / 128 : 0;
+  int32_t* status = at<int32_t>(ws, L.status);
+
+  // ---- gate/up + SwiGLU ---------------------------------------------------
+  {
+    const int BN = (2 * I) % 256 == 0 ? 256 : 128;
+    GemmMaps m;
+    bool ok = make_map_bf16(&m.a_r, 2, xperm, d64, rows, 1, d64 * 2, 0, 128) &&
+              make_map_bf16(&m.b_r, 3, W13, d64, 2 * I64, n, d64 * 2, 2 * I64 * d64 * 2, BN);
+    if (ns > 0) {
+      ok = ok && make_map_bf16(&m.a_s, 2, u, d64, T, 1, d64 * 2, 0, 128) &&
+           make_map_bf16(&m.b_s, 3, W13_s, d64, 2 * I64 * ns, 1, d64 * 2, 2 * I64 * ns * d64 * 2,
+                         BN);
+    } else {
+      m.a_s = m.a_r;
+      m.b_s = m.b_r;
+    }
+    if (!ok) return MOE_ERR_CUDA;
+    GroupedGemmArgs a{};
+    a.offsets = offsets;
+    a.n_routed = n;
+    a.shared_rows = ns > 0 ? static_cast<int32_t>(T) : 0;
+    a.kb_routed = d / 64;
+    a.kb_shared = d / 64;
+    a.kb_per_expert = d / 64;
+    a.nt_routed = 2 * I / BN;
+    a.nt_shared = 2 * I * ns / BN;
+    a.out_r = act;
+    a.ld_r = I;
+    a.out_s = act_s;
+    a.ld_s = static_cast<int64_t>(I) * ns;
+    a.status = status;
+    const int64_t tiles = routed_mt_ub * a.nt_routed + shared_mt * a.nt_shared;
+    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    Stage sg(MOE_KERNEL_GEMM_GATE_UP, st);
+    if (int rc = launch_grouped_gemm(BN, kEpiSwiGLU, m, a, grid, st)) return rc;
+  }
+  // ---- down projection ----------------------------------------------------
+  {
+    const int BN = d % 256 == 0 ? 256 : (d % 128 == 0 ? 128 : 64);
+    GemmMaps m;
+    bool ok = make_map_bf16(&m.a_r, 2, act, I64, rows, 1, I64 * 2, 0, 128) &&
+              make_map_bf16(&m.b_r, 3, W2, I64, d64, n, I64 * 2, d64 * I64 * 2, BN);
+    if (ns > 0) {
+      ok = ok && make_map_bf16(&m.a_s, 2, act_s, I64 * ns, T, 1, I64 * ns * 2, 0, 128) &&
+           make_map_bf16(&m.b_s, 3, W2_s, I64, d64, ns, I64 * 2, d64 * I64 * 2, BN);
+    } else {
+      m.a_s = m.a_r;
+      m.b_s = m.b_r;
+    }
+    if (!ok) return MOE_ERR_CUDA;
+    GroupedGemmArgs a{};
+    a.offsets = offsets;
+    a.n_routed = n;
+    a.shared_rows = ns > 0 ? static_cast<int32_t>(T) : 0;
+    a.kb_routed = I / 64;
+    a.kb_shared = I * ns / 64;
+    a.kb_per_expert = I / 64;
+    a.nt_routed = d / BN;
+    a.nt_shared = d / BN;
+    a.out_r = y;
+    a.ld_r = d;
+    a.out_s = ysh;
+    a.ld_s = d;
+    a.status = status;
+    const int64_t tiles = routed_mt_ub * a.nt_routed + shared_mt * a.nt_shared;
+    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+    Stage sg(MOE_KERNEL_GEMM_DOWN, st);
+    if (int rc = launch_grouped_gemm(BN, kEpiPlain, m, a, grid, st)) return rc;
+  }
+  return MOE_OK;
+}
+
+int forward_device(const moe_shape_t& s, const Layout& L, const void* u, const void* E,
+                   const float* bias, const void* W13, const void* W2, const void* W13_s,
+                   const void* W2_s, void* h, void* ws, cudaStream_t st, int sms) {
+  const int64_t T = s.T;
+  const int K = s.top_k, n = s.n_routed;
+  int32_t* idx = at<int32_t>(ws, L.idx);
+  float* w = at<float>(ws, L.w);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  void* y = at<void>(ws, L.y);
+  float* ysh = at<float>(ws, L.ysh);
+  {
+    Stage sg(MOE_KERNEL_ROUTER, st);
+    if (int rc = launch_router(s.dtype, u, E, bias, T, s.d, n, K, s.flags, idx, w, nullptr, st))
+      return rc;
+  }
+  {
+    Stage sg(MOE_KERNEL_DISPATCH, st);
+    if (int rc = launch_dispatch(idx, T, K, n, at<int32_t>(ws, L.chunk_counts),
+                                 at<int32_t>(ws, L.chunk_base), counts, offsets, perm, inv, st))
+      return rc;
+  }
+  if (int rc = run_expert_ffn(s, L, u, perm, offsets, W13, W2, W13_s, W2_s, y, ysh, ws, st, sms))
+    return rc;
+  Stage sg(MOE_KERNEL_COMBINE, st);
+  return launch_combine(s.dtype, u, ysh, y, w, inv, T, s.d, K, h, st);
+}
+
+bool shared_ptrs_ok(const moe_shape_t& s, const void* W13_s, const void* W2_s) {
+  return s.n_shared == 0 || (W13_s && W2_s);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_strerror(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_NULLPTR: return "null pointer";
+    case MOE_ERR_SHAPE: return "invalid shape";
+    case MOE_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_DTYPE: return "invalid dtype";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_CHECK: return "a kernel gave up waiting (device check)";
+    case MOE_ERR_UNSUPPORTED: return "device is not sm_100 (B200)";
+    default: return "unknown status";
+  }
+}
+
+const char* moe_version(void) { return "moe-b200 0.1.0 (sm_100a)"; }
+
+uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+int moe_profile_enable(int on) {
+  prof().on.store(on != 0);
+  return MOE_OK;
+}
+
+int moe_profile_read(int32_t* kinds, float* ms, int32_t max, int32_t* count) {
+  if (!count || (max > 0 && (!kinds || !ms))) return MOE_ERR_NULLPTR;
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> lock(p.mu);
+  int32_t n = 0;
+  int rc = MOE_OK;
+  for (const ProfRec& r : p.recs) {
+    if (n < max) {
+      float t = 0.0f;
+      if (cudaEventSynchronize(r.end) != cudaSuccess ||
+          cudaEventElapsedTime(&t, r.beg, r.end) != cudaSuccess)
+        rc = MOE_ERR_CUDA;
+      kinds[n] = r.kind;
+      ms[n] = t;
+      ++n;
+    }
+    p.pool.push_back(r.beg);
+    p.pool.push_back(r.end);
+  }
+  p.recs.clear();
+  *count = n;
+  return rc;
+}
+
+const char* moe_kernel_name(int32_t kind) {
+  switch (kind) {
+    case MOE_KERNEL_ROUTER: return "router_topk";
+    case MOE_KERNEL_DISPATCH: return "dispatch";
+    case MOE_KERNEL_GATHER: return "gather_rows";
+    case MOE_KERNEL_GEMM_GATE_UP: return "grouped_gemm_gate_up_swiglu";
+    case MOE_KERNEL_GEMM_DOWN: return "grouped_gemm_down";
+    case MOE_KERNEL_COMBINE: return "combine_residual";
+    case MOE_KERNEL_FFN_F32: return "ffn_f32";
+    case MOE_KERNEL_MEMSET: return "memset";
+    case MOE_KERNEL_PACK: return "pack_w13";
+    case MOE_KERNEL_BALANCE: return "expert_balance";
+    default: return "unknown";
+  }
+}
+
+int moe_workspace_size(const moe_shape_t* shape, size_t* bytes) {
+  if (!bytes) return MOE_ERR_NULLPTR;
+  if (int rc = validate(shape)) return rc;
+  *bytes = layout_of(*shape).total;
+  return MOE_OK;
+}
+
+int moe_workspace_size_host(const moe_shape_t* shape, size_t* bytes) {
+  if (!bytes) return MOE_ERR_NULLPTR;
+  if (int rc = validate(shape)) return rc;
+  *bytes = layout_of(*shape).total_host;
+  return MOE_OK;
+}
+
+int moe_pack_w13(const moe_shape_t* shape, int32_t n_experts, const void* W1, const void* W3,
+                 void* W13, moe_stream_t stream) {
+  if (int rc = validate(shape)) return rc;
+  if (n_experts < 0) return MOE_ERR_SHAPE;
+  if (n_experts == 0) return MOE_OK;
+  if (!W1 || !W3 || !W13) return MOE_ERR_NULLPTR;
+  if (misaligned(W1) || misaligned(W3) || misaligned(W13)) return MOE_ERR_ALIGN;
+  DeviceInfo di;
+  if (int rc = device_info(&di)) return rc;
+  Stage sg(MOE_KERNEL_PACK, static_cast<cudaStream_t>(stream));
+  return launch_pack_w13(shape->dtype, W1, W3, W13, n_experts, shape->inter, shape->d,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int moe_route(const moe_shape_t* shape, const void* u, const void* E, const float* bias,
+              int32_t* idx, float* w, moe_stream_t stream) {
+  if (int rc = validate(shape)) return rc;
+  if (shape->T == 0) return MOE_OK;
+  if (!u || !E || !idx || !w) return MOE_ERR_NULLPTR;
+  if (misaligned(u) || misaligned(E) || misaligned(idx) || misaligned(w) ||
+      (bias && misaligned(bias)))
+    return MOE_ERR_ALIGN;
+  DeviceInfo di;
+  if (int rc = device_info(&di)) return rc;
+  Stage sg(MOE_KERNEL_ROUTER, static_cast<cudaStream_t>(stream));
+  return launch_router(shape->dtype, u, E, bias, shape->T, shape->d, shape->n_routed,
+                       shape->top_k, shape->flags, idx, w, nullptr,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int moe_dispatch(const moe_shape_t* shape, const int32_t* idx, int32_t* counts, int32_t* offsets,
+                 int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (int rc = validate(shape)) return rc;
+  if (!counts || !offsets || !ws) return MOE_ERR_NULLPTR;
+  if (shape->T > 0 && (!idx || !perm || !inv)) return MOE_ERR_NULLPTR;
+  if (misaligned(counts) || misaligned(offsets) || misaligned(ws) ||
+      (shape->T > 0 && (misaligned(idx) || misaligned(perm) || misaligned(inv))))
+    return MOE_ERR_ALIGN;
+  const Layout L = layout_of(*shape);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  DeviceInfo di;
+  if (int rc = device_info(&di)) return rc;
+  Stage sg(MOE_KERNEL_DISPATCH, static_cast<cudaStream_t>(stream));
+  return launch_dispatch(idx, shape->T, shape->top_k, shape->n_routed,
+                         at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.chunk_base), counts,
+                         offsets, perm, inv, static_cast<cudaStream_t>(stream));
+}
+
+int moe_expert_ffn(const moe_shape_t* shape, const void* u, const int32_t* perm,
+                   const int32_t* offsets, const void* W13, const void* W2, const void* W13_s,
+                   const void* W2_s, void* y, float* ysh, void* ws, size_t ws_bytes,
+                   moe_stream_t stream) {
+  if (int rc = validate(shape)) return rc;
+  if (shape->T == 0) return MOE_OK;
+  if (!u || !perm || !offsets || !W13 || !W2 || !y || !ysh || !ws) return MOE_ERR_NULLPTR;
+  if (!shared_ptrs_ok(*shape, W13_s, W2_s)) return MOE_ERR_NULLPTR;
+  if (misaligned(u) || misaligned(perm) || misaligned(offsets) || misaligned(W13) ||
+      misaligned(W2) || misaligned(y) || misaligned(ysh) || misaligned(ws) ||
+      (W13_s && misaligned(W13_s)) || (W2_s && misaligned(W2_s)))
+    return MOE_ERR_ALIGN;
+  const Layout L = layout_of(*shape);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  DeviceInfo di;
+  if (int rc = device_info(&di)) return rc;
+  return run_expert_ffn(*shape, L, u, perm, offsets, W13, W2, W13_s, W2_s, y, ysh, ws,
+                        static_cast<cudaStream_t>(stream), di.sms);
+}
+
+int moe_combine(const moe_shape_t* shape, const void* u, const float* ysh, const void* y,
+                const float* w, const int32_t* inv, void* h, moe_stream_t stream) {
+  if (int rc = validate(shape)) return rc;
+  if (shape->T == 0) return MOE_OK;
+  if (!u || !ysh || !y || !w || !inv || !h) return MOE_ERR_NULLPTR;
+  if (misaligned(u) || misaligned(ysh) || misaligned(y) || misaligned(w) || misaligned(inv) ||
+      misaligned(h))
+    return MOE_ERR_ALIGN;
+  DeviceInfo di;
+  if (int rc = device_info(&di)) return rc;
+  Stage sg(MOE_KERNEL_COMBINE, static_cast<cudaStream_t>(stream));
+  return launch_combine(shape->dtype, u, ysh, y, w, inv, shape->T, shape->d, shape->top_k, h,
+                        static_cast<cudaStream_t>(stream));
+}
+
+int moe_layer_forward(const moe_shape_t* shape, const void* u, const void* E, const float* bias,
+                      const void* W13, const void* W2, const void* W13_s, const void* W2_s,
+                      void* h, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (int rc = validate(shape)) return rc;
+  if (shape->T == 0) return MOE_OK;
+  if (!u || !E || !W13 || !W2 || !h || !ws) return MOE_ERR_NULLPTR;
+  if (!shared_ptrs_ok(*shape, W13_s, W2_s)) return MOE_ERR_NULLPTR;
+  if (misaligned(u) || misaligned(E) || misaligned(W13) || misaligned(W2) || misaligned(h) ||
+      misaligned(ws) || (bias && misaligned(bias)) || (W13_s && misaligned(W13_s)) ||
+      (W2_s && misaligned(W2_s)))
+    return MOE_ERR_ALIGN;
+  const Layout L = layout_of(*shape);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  DeviceInfo di;
+  if (int rc = device_info(&di)) return rc;
+  return forward_device(*shape, L, u, E, bias, W13, W2, W13_s, W2_s, h, ws,
+                        static_cast<cudaStream_t>(stream), di.sms);
+}
+
+int moe_layer_forward_host(const moe_shape_t* shape, const void* u_host, const void* E,
+                           const float* bias, const void* W13, const void* W2, const void* W13_s,
+                           const void* W2_s, void* h_host, void* ws, size_t ws_bytes,
+                           moe_stream_t stream) {
+  if (int rc = validate(shape)) return rc;
+  if (shape->T == 0) return MOE_OK;
+  if (!u_host || !E || !W13 || !W2 || !h_host || !ws) return MOE_ERR_NULLPTR;
+  if (!shared_ptrs_ok(*shape, W13_s, W2_s)) return MOE_ERR_NULLPTR;
+  if (misaligned(E) || misaligned(W13) || misaligned(W2) || misaligned(ws) ||
+      (bias && misaligned(bias)) || (W13_s && misaligned(W13_s)) || (W2_s && misaligned(W2_s)))
+    return MOE_ERR_ALIGN;
+  const Layout L = layout_of(*shape);
+  if (ws_bytes < L.total_host) return MOE_ERR_WORKSPACE;
+  DeviceInfo di;
+  if (int rc = device_info(&di)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(shape->T) * shape->d * elem_bytes(shape->dtype);
+  void* u_dev = at<void>(ws, L.u_host);
+  void* h_dev = at<void>(ws, L.h_host);
+  if (cudaMemcpyAsync(u_dev, u_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (int rc = forward_device(*shape, L, u_dev, E, bias, W13, W2, W13_s, W2_s, h_dev, ws, st,
+                              di.sms))
+    return rc;
+  if (cudaMemcpyAsync(h_host, h_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_expert_balance(const moe_shape_t* shape, const void* u, const void* E, const float* bias,
+                       const int32_t* counts, float* f, float* P, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  if (int rc = validate(shape)) return rc;
+  if (shape->T == 0) return MOE_ERR_SHAPE;  // eqs. (12)-(13) divide by T
+  if (!u || !E || !counts || !f || !P || !ws) return MOE_ERR_NULLPTR;
+  if (misaligned(u) || misaligned(E) || misaligned(ws) || (bias && misaligned(bias)))
+    return MOE_ERR_ALIGN;
+  const Layout L = layout_of(*shape);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  DeviceInfo di;
+  if (int rc = device_info(&di)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Stage sg(MOE_KERNEL_BALANCE, st);
+  float* pstat = at<float>(ws, L.pstat);
+  // the router pass also rewrites the workspace's idx / w scratch
+  if (int rc = launch_router(shape->dtype, u, E, bias, shape->T, shape->d, shape->n_routed,
+                             shape->top_k, shape->flags, at<int32_t>(ws, L.idx), at<float>(ws, L.w),
+                             pstat, st))
+    return rc;
+  return launch_balance_reduce(pstat, router_num_ctas(shape->T), counts, shape->T,
+                               shape->n_routed, shape->top_k, f, P, st);
+}
+
+int moe_read_status(const void* ws, int32_t* status, moe_stream_t stream) {
+  if (!ws || !status) return MOE_ERR_NULLPTR;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* dev = reinterpret_cast<int32_t*>(const_cast<void*>(ws));
+  if (cudaMemcpyAsync(status, dev, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(dev, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

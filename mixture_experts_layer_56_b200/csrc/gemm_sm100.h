@@ -1,0 +1,45 @@
+// Host interface of the tcgen05 grouped expert GEMM (gemm_sm100.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+namespace sm100 {
+
+enum { kEpiSwiGLU = 0, kEpiPlain = 1 };
+
+// One launch covers the shared-expert group (when shared_rows > 0) and the
+// n_routed routed groups whose rows are offsets[e] .. offsets[e+1]-1.
+struct GroupedGemmArgs {
+  const int32_t* offsets;  // device, [n_routed + 1]
+  int32_t n_routed;
+  int32_t shared_rows;     // rows of the shared group (T) or 0
+  int32_t kb_routed;       // 64-wide k-blocks of a routed tile
+  int32_t kb_shared;       // 64-wide k-blocks of a shared tile
+  int32_t kb_per_expert;   // B's third coordinate advances every kb_per_expert k-blocks
+  int32_t nt_routed;       // BN-wide N tiles per routed group
+  int32_t nt_shared;       // BN-wide N tiles of the shared group
+  void* out_r;             // routed output (bf16), row stride ld_r elements
+  int64_t ld_r;
+  void* out_s;             // shared output: bf16 (SwiGLU) or fp32 (plain)
+  int64_t ld_s;
+  int32_t* status;         // workspace status word
+};
+
+// A maps: rank 2 {K, rows}; B maps: rank 3 {K, N rows, experts}; bf16, box
+// {64, 128 (A) or BN (B)}, 128-byte swizzle.
+struct GemmMaps {
+  CUtensorMap a_r, a_s, b_r, b_s;
+};
+
+bool make_map_bf16(CUtensorMap* map, int rank, const void* base, uint64_t inner, uint64_t rows,
+                   uint64_t depth, uint64_t row_stride_bytes, uint64_t depth_stride_bytes,
+                   uint32_t box_rows);
+
+int launch_grouped_gemm(int BN, int epi, const GemmMaps& maps, const GroupedGemmArgs& args,
+                        int grid, cudaStream_t stream);
+
+}  // namespace sm100
+}  // namespace moe

@@ -1,0 +1,42 @@
+// Launch wrappers of the non-GEMM kernels of libmoe (host interface).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kDispatchChunk = 256;  // tokens per dispatch block
+
+inline int64_t dispatch_num_chunks(int64_t T) { return (T + kDispatchChunk - 1) / kDispatchChunk; }
+int router_num_ctas(int64_t T);
+
+int launch_router(int dtype, const void* u, const void* E, const float* bias, int64_t T, int d,
+                  int n, int K, int flags, int32_t* idx, float* w, float* pstat,
+                  cudaStream_t st);
+
+int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_counts,
+                    int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* perm,
+                    int32_t* inv, cudaStream_t st);
+
+int launch_gather(int dtype, const void* u, const int32_t* perm, int64_t rows, int d, int K,
+                  void* xperm, cudaStream_t st);
+
+int launch_combine(int dtype, const void* u, const float* ysh, const void* y, const float* w,
+                   const int32_t* inv, int64_t T, int d, int K, void* h, cudaStream_t st);
+
+int launch_pack_w13(int dtype, const void* W1, const void* W3, void* W13, int n_experts, int I,
+                    int d, cudaStream_t st);
+
+// fp32 expert FFN on CUDA cores (the MOE_DTYPE_F32 path)
+int launch_ffn_f32(const float* xperm, const float* u, const int32_t* offsets, int n_routed,
+                   int64_t T, int n_shared, int d, int I, const float* W13, const float* W2,
+                   const float* W13_s, const float* W2_s, float* act, float* act_s, float* y,
+                   float* ysh, int max_routed_mtiles, cudaStream_t st);
+
+int launch_balance_reduce(const float* pstat, int nblocks, const int32_t* counts, int64_t T,
+                          int n, int K, float* f, float* P, cudaStream_t st);
+
+int launch_zero(void* p, size_t bytes, cudaStream_t st);
+
+}  // namespace moe

@@ -38,7 +38,7 @@ import numpy as np
 # router: eqs. (10)-(11)
 # --------------------------------------------------------------------------
 def router_logits(u: np.ndarray, E: np.ndarray, bias: np.ndarray | None = None,
-                  block: int = 2048) -> np.ndarray:
+                  block: int | None = None) -> np.ndarray:
     """l[t, i] = u_t^T e_i (+ b_i), eq. (11) before the softmax.
 
     One matrix-vector product per expert i (over blocks of tokens), so that
@@ -46,6 +46,8 @@ def router_logits(u: np.ndarray, E: np.ndarray, bias: np.ndarray | None = None,
     """
     T = u.shape[0]
     n = E.shape[0]
+    if block is None:
+        block = max(1, (1 << 21) // max(1, u.shape[1]))
     l = np.empty((T, n), dtype=np.float64)
     for t0 in range(0, T, block):
         ub = u[t0:t0 + block]
@@ -186,15 +188,27 @@ def layer_forward(u, E, bias, W1, W3, W2, W1_s, W3_s, W2_s, K,
 
 def layer_forward_tokens(u, idx, g, tokens, W1, W3, W2, W1_s, W3_s, W2_s):
     """h for the listed tokens only, given each token's routing (idx, g):
-    eq. (9) evaluated one token at a time (for sampled checks at full size)."""
+    eq. (9) for those tokens (for sampled checks at full size).  The routed
+    sum is taken expert by expert over the sampled tokens that chose it."""
     tokens = np.asarray(tokens, dtype=np.int64)
     x = u[tokens]
     h = x + shared_experts(x, W1_s, W3_s, W2_s)
-    for j, t in enumerate(tokens):
-        for k in range(idx.shape[1]):
-            e = int(idx[t, k])
-            h[j] += g[t, k] * swiglu_ffn(x[j:j + 1], W1[e], W3[e], W2[e])[0]
+    sel = np.asarray(idx)[tokens]
+    gs = np.asarray(g)[tokens]
+    for e in np.unique(sel):
+        rows, ks = np.nonzero(sel == e)
+        h[rows] += gs[rows, ks][:, None] * swiglu_ffn(x[rows], W1[e], W3[e], W2[e])
     return h
+
+
+def topk_gates_select_only_bias(l: np.ndarray, bias: np.ndarray, K: int):
+    """Bias that steers only the selection: the K largest l + b are chosen
+    (lower index first on ties) and the gates are the softmax of the
+    unbiased logits l at those experts, not renormalised."""
+    order = np.argsort(-(l + np.asarray(bias, dtype=np.float64)[None, :]), axis=1,
+                       kind="stable")[:, :K]
+    s = softmax(l)
+    return order.astype(np.int32), np.take_along_axis(s, order, axis=1)
 
 
 # --------------------------------------------------------------------------

@@ -1,0 +1,204 @@
+"""Helpers of the GPU parity tests: run every stage of the layer through the C
+ABI and compare it with the CPU oracle on the same seeded inputs.
+
+Bars (the layer's floating-point results are bf16 with fp32 accumulation):
+* routing indices, per-expert counts, offsets, the permutation and its
+  inverse: bit-exact.  A token whose oracle scores have two of their K+1
+  largest values closer than TIE_GAP is a near tie: it is counted and its
+  selection only has to be a valid top-K of the oracle's scores within
+  TIE_GAP.  Dispatch outputs are compared with the oracle's dispatch of the
+  GPU's own routing, so they stay bit-exact on near ties too.
+* gates: |w - s| <= 1e-6 + 1e-5 s (fp32 softmax).
+* bf16 tensors: |x - x_ref| <= 2e-2 + 2^-8 |x_ref| elementwise (the second
+  term is the bf16 output rounding, which alone exceeds 2e-2 once |x| > 5.12)
+  and ||x - x_ref||_F / ||x_ref||_F <= 1e-2.
+* fp32 layer: |x - x_ref| <= 1e-4 + 1e-5 |x_ref|, relative Frobenius <= 1e-5.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from mixture_experts_layer_56_b200 import _lib as L
+from mixture_experts_layer_56_b200 import synthetic as S
+from mixture_experts_layer_56_b200.layer import MoELayer, to_device, to_numpy
+from oracle import moe_oracle as O
+
+TIE_GAP = 1e-5
+NAMES = ("u", "E", "bias", "W1", "W3", "W2", "W1_s", "W3_s", "W2_s")
+
+
+def f64_inputs(x: S.LayerInputs) -> dict:
+    return {k: x.as_f64(k) for k in NAMES}
+
+
+def as_f64(t: torch.Tensor) -> np.ndarray:
+    a = to_numpy(t)
+    if a.dtype == np.uint16:
+        return S.bf16_bits_to_f32(a).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def gpu_stages(x: S.LayerInputs, device="cuda:0", flags=0, layer=None):
+    """Every stage through the C ABI, plus the fused moe_layer_forward."""
+    wl = x.wl
+    T, K, n, d = wl.T, wl.top_k, wl.n_routed, wl.d
+    layer = layer or MoELayer(x, device, flags=flags)
+    sh = layer.shape
+    dev = layer.device
+    u = to_device(x.u, dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+    idx = torch.full((T, K), -1, **i32)
+    w = torch.full((T, K), -1.0, dtype=torch.float32, device=dev)
+    L.moe_route(sh, u, layer.E, layer.bias, idx, w)
+    counts = torch.full((n,), -1, **i32)
+    offsets = torch.full((n + 1,), -1, **i32)
+    perm = torch.full((T * K,), -1, **i32)
+    inv = torch.full((T * K,), -1, **i32)
+    L.moe_dispatch(sh, idx, counts, offsets, perm, inv, layer.ws)
+    y = torch.full((T * K, d), float("nan"), dtype=layer.elem_dtype, device=dev)
+    ysh = torch.full((T, d), float("nan"), dtype=torch.float32, device=dev)
+    L.moe_expert_ffn(sh, u, perm, offsets, layer.W13, layer.W2, layer.W13_s, layer.W2_s, y, ysh,
+                     layer.ws)
+    h = torch.full_like(u, float("nan"))
+    L.moe_combine(sh, u, ysh, y, w, inv, h)
+    h_fwd = layer.forward(u)
+    torch.cuda.synchronize()
+    status = layer.status()
+    return dict(idx=to_numpy(idx), w=to_numpy(w), counts=to_numpy(counts),
+                offsets=to_numpy(offsets), perm=to_numpy(perm), inv=to_numpy(inv),
+                y=as_f64(y), ysh=as_f64(ysh), h=as_f64(h), h_raw=to_numpy(h),
+                h_fwd_raw=to_numpy(h_fwd), status=status, layer=layer)
+
+
+def near_tie_tokens(s: np.ndarray, K: int) -> np.ndarray:
+    """Tokens whose K+1 largest scores hold two values closer than TIE_GAP."""
+    m = min(K + 1, s.shape[1])
+    top = -np.sort(-s, axis=1)[:, :m]
+    if m < 2:
+        return np.zeros(s.shape[0], dtype=bool)
+    return np.min(top[:, :-1] - top[:, 1:], axis=1) < TIE_GAP
+
+
+def check_routing(idx: np.ndarray, w: np.ndarray, s: np.ndarray, K: int,
+                  ref_idx: np.ndarray | None = None, gate_s: np.ndarray | None = None):
+    """Returns (near-tie count, mismatch count); asserts the bars above.
+    ``s`` ranks the experts (the selection key), ``gate_s`` gives the gates
+    (defaults to s)."""
+    gate_s = s if gate_s is None else gate_s
+    if ref_idx is None:
+        ref_idx, _ = O.topk_gates(s, K)
+    near = near_tie_tokens(s, K)
+    mism = np.any(idx != ref_idx, axis=1)
+    bad = np.where(mism & ~near)[0]
+    assert bad.size == 0, f"{bad.size} tokens differ outside near ties, e.g. t={bad[:5]}"
+    n = s.shape[1]
+    assert np.all((idx >= 0) & (idx < n))
+    for t in np.where(mism)[0]:
+        sel = idx[t]
+        assert len(set(sel.tolist())) == K
+        kth = np.sort(s[t])[::-1][K - 1]
+        assert np.all(s[t, sel] >= kth - TIE_GAP)
+        assert np.all(np.diff(s[t, sel]) <= TIE_GAP)
+    g = np.take_along_axis(gate_s, idx.astype(np.int64), axis=1)
+    err = np.abs(w.astype(np.float64) - g)
+    assert np.all(err <= 1e-6 + 1e-5 * g), float(err.max())
+    return int(near.sum()), int(mism.sum())
+
+
+def check_dispatch(gpu: dict, n: int):
+    counts, offsets, perm, inv = O.dispatch(gpu["idx"], n)
+    np.testing.assert_array_equal(gpu["counts"], counts)
+    np.testing.assert_array_equal(gpu["offsets"], offsets)
+    np.testing.assert_array_equal(gpu["perm"], perm)
+    np.testing.assert_array_equal(gpu["inv"], inv)
+
+
+def assert_close(got: np.ndarray, ref: np.ndarray, what: str, bf16: bool = True):
+    if bf16:
+        atol, rtol_el, rel_fro = 2e-2, 2.0 ** -8, 1e-2
+    else:
+        atol, rtol_el, rel_fro = 1e-4, 1e-5, 1e-5
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - ref)
+    bound = atol + rtol_el * np.abs(ref)
+    worst = int(np.argmax(err - bound))
+    assert np.all(err <= bound), (f"{what}: max |err| {err.max():.3e} (at {worst}: got "
+                                  f"{got.flat[worst]:.6f}, ref {ref.flat[worst]:.6f})")
+    nref = np.linalg.norm(ref)
+    if nref > 0:
+        rel = np.linalg.norm(got - ref) / nref
+        assert rel <= rel_fro, f"{what}: relative Frobenius error {rel:.3e}"
+    return float(err.max())
+
+
+def full_parity(x: S.LayerInputs, flags: int = 0, device="cuda:0"):
+    """Every stage against the oracle, every token.  Returns a report."""
+    wl = x.wl
+    f = f64_inputs(x)
+    gpu = gpu_stages(x, device, flags)
+    assert gpu["status"] == 0
+    bf16 = wl.dtype == S.DTYPE_BF16
+    l = O.router_logits(f["u"], f["E"], None)
+    if flags & L.MOE_FLAG_BIAS_SELECT_ONLY and f["bias"] is not None:
+        key = O.softmax(l + f["bias"][None, :])
+        gate_s = O.softmax(l)
+        ref_idx, _ = O.topk_gates_select_only_bias(l, f["bias"], wl.top_k)
+    else:
+        key = O.softmax(l if f["bias"] is None else l + f["bias"][None, :])
+        gate_s = key
+        ref_idx = None
+    near, mism = check_routing(gpu["idx"], gpu["w"], key, wl.top_k, ref_idx, gate_s)
+    check_dispatch(gpu, wl.n_routed)
+    # FFN + combine evaluated by the oracle on the GPU's routing
+    ref = O.layer_forward(f["u"], f["E"], f["bias"], f["W1"], f["W3"], f["W2"], f["W1_s"],
+                          f["W3_s"], f["W2_s"], wl.top_k, idx=gpu["idx"])
+    g = np.take_along_axis(gate_s, gpu["idx"].astype(np.int64), axis=1)
+    ref_h = O.combine(f["u"], ref["y_shared"], ref["y"], g, ref["inv"], wl.top_k)
+    ey = assert_close(gpu["y"], ref["y"], "y", bf16)
+    esh = assert_close(gpu["ysh"], ref["y_shared"], "ysh", bf16)
+    eh = assert_close(gpu["h"], ref_h, "h", bf16)
+    assert np.array_equal(gpu["h_raw"], gpu["h_fwd_raw"]), "layer_forward != stage-wise result"
+    return dict(near_ties=near, mismatches=mism, err_y=ey, err_ysh=esh, err_h=eh, gpu=gpu)
+
+
+def sample_tokens(gpu: dict, K: int, n_random: int = 512, seed: int = 0) -> np.ndarray:
+    """Random tokens plus every token of the most-loaded expert's first tile
+    and of each expert's last partial 128-row tile."""
+    T = gpu["idx"].shape[0]
+    rng = np.random.default_rng(seed)
+    picks = set(rng.choice(T, size=min(n_random, T), replace=False).tolist())
+    counts, offsets, perm = gpu["counts"], gpu["offsets"], gpu["perm"]
+    e_max = int(np.argmax(counts))
+    for p in range(offsets[e_max], min(offsets[e_max] + 128, offsets[e_max + 1])):
+        picks.add(int(perm[p]) // K)
+    for e in range(counts.size):
+        c = int(counts[e])
+        if c % 128:
+            for p in range(offsets[e] + (c // 128) * 128, offsets[e + 1]):
+                picks.add(int(perm[p]) // K)
+    return np.array(sorted(picks), dtype=np.int64)
+
+
+def sampled_parity(x: S.LayerInputs, device="cuda:0", n_random: int = 512):
+    """Full-size check: routing and dispatch for every token, y and h on a
+    sample of tokens (see sample_tokens)."""
+    wl = x.wl
+    f = f64_inputs(x)
+    gpu = gpu_stages(x, device)
+    assert gpu["status"] == 0
+    l = O.router_logits(f["u"], f["E"], f["bias"])
+    s = O.softmax(l)
+    near, mism = check_routing(gpu["idx"], gpu["w"], s, wl.top_k)
+    check_dispatch(gpu, wl.n_routed)
+    toks = sample_tokens(gpu, wl.top_k, n_random)
+    g = np.take_along_axis(s, gpu["idx"].astype(np.int64), axis=1)
+    ref_h = O.layer_forward_tokens(f["u"], gpu["idx"], g, toks, f["W1"], f["W3"], f["W2"],
+                                   f["W1_s"], f["W3_s"], f["W2_s"])
+    eh = assert_close(gpu["h"][toks], ref_h, "h (sampled)")
+    # shared output on the sample
+    ref_sh = O.shared_experts(f["u"][toks], f["W1_s"], f["W3_s"], f["W2_s"])
+    esh = assert_close(gpu["ysh"][toks], ref_sh, "ysh (sampled)")
+    assert np.array_equal(gpu["h_raw"], gpu["h_fwd_raw"]), "layer_forward != stage-wise result"
+    return dict(near_ties=near, mismatches=mism, err_h=eh, err_ysh=esh, sampled=int(toks.size),
+                gpu=gpu)

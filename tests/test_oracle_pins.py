@@ -350,3 +350,20 @@ def test_expert_balance_statistics():
     np.testing.assert_allclose(fd, [1.0, 1.0])
     np.testing.assert_allclose(Pd, [0.5, 0.5])
     np.testing.assert_allclose(Ld, 2.0)
+
+
+def test_select_only_bias_variant():
+    """Bias that steers only the selection: with b = 0 it is the plain top-K;
+    with a large bias on one expert that expert is always chosen while its
+    gate stays its unbiased softmax score."""
+    rng = np.random.default_rng(17)
+    l = _rand(rng, 40, 8)
+    i0, g0 = O.topk_gates_select_only_bias(l, np.zeros(8), 3)
+    i1, g1 = O.topk_gates(O.softmax(l), 3)
+    np.testing.assert_array_equal(i0, i1)
+    np.testing.assert_array_equal(g0, g1)
+    b = np.zeros(8)
+    b[5] = 1e3
+    i2, g2 = O.topk_gates_select_only_bias(l, b, 3)
+    assert np.all(i2[:, 0] == 5)
+    np.testing.assert_allclose(g2[:, 0], scipy.special.softmax(l, axis=1)[:, 5], rtol=1e-14)
