@@ -60,6 +60,18 @@ def weight_bytes_streamed(wl, counts):
     return (hit + wl.n_shared) * 3 * wl.d * wl.inter * el + wl.n_routed * wl.d * el
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest value of x over all ranks (x itself without a process
+    group): the job's time is its slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
     """Polls the SM clock and the clock-event reasons (read only) during the
@@ -272,11 +284,7 @@ def run_ours(args):
         barrier()
     launches = L.moe_launch_count() - launches0
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     assert layer.status() == 0
     tokens = wl.T * world * args.steps
     value = tokens / (total_ms / 1e3)
@@ -310,11 +318,7 @@ def run_ours(args):
         layer.forward_host(u_h, h_h, stream=stream)
     e_end.record(stream)
     barrier()
-    e2e_ms = e_start.elapsed_time(e_end)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
     e2e_value = wl.T * world * e2e_steps / (e2e_ms / 1e3)
     io_bytes = wl.T * wl.d * (2 if wl.dtype == "bf16" else 4)
 

@@ -77,6 +77,7 @@ dispatch_scan_kernel(const int32_t* __restrict__ chunk_counts, int64_t nchunks, 
   __shared__ int tot[256];
   __shared__ int off[257];
   const int e = threadIdx.x;
+  // pass 1: tokens per expert (loads batched so that 8 are in flight)
   int run = 0;
   if (e < n) {
     int64_t c = 0;
@@ -85,16 +86,9 @@ dispatch_scan_kernel(const int32_t* __restrict__ chunk_counts, int64_t nchunks, 
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = chunk_counts[(c + i) * n + e];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        chunk_base[(c + i) * n + e] = run;
-        run += v[i];
-      }
+      for (int i = 0; i < 8; ++i) run += v[i];
     }
-    for (; c < nchunks; ++c) {
-      const int v = chunk_counts[c * n + e];
-      chunk_base[c * n + e] = run;
-      run += v;
-    }
+    for (; c < nchunks; ++c) run += chunk_counts[c * n + e];
     counts[e] = run;
   }
   tot[e] = e < n ? run : 0;
@@ -112,15 +106,30 @@ dispatch_scan_kernel(const int32_t* __restrict__ chunk_counts, int64_t nchunks, 
   off[e + 1] = x;
   if (e == 0) off[0] = 0;
   __syncthreads();
+  // pass 2: where each chunk's tokens of expert e start
   if (e < n) {
-    const int base = off[e];
+    int base = off[e];
     offsets[e] = base;
-    for (int64_t c = 0; c < nchunks; ++c) chunk_base[c * n + e] += base;
+    int64_t c = 0;
+    for (; c + 8 <= nchunks; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = chunk_counts[(c + i) * n + e];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        chunk_base[(c + i) * n + e] = base;
+        base += v[i];
+      }
+    }
+    for (; c < nchunks; ++c) {
+      chunk_base[c * n + e] = base;
+      base += chunk_counts[c * n + e];
+    }
   }
   if (e == 0) offsets[n] = off[n];
 }
 
-template <int NW>
+template <int NW, int KMAX>
 __global__ void __launch_bounds__(kDispThreads)
 dispatch_scatter_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n,
                         const int32_t* __restrict__ chunk_base, int32_t* __restrict__ perm,
@@ -128,8 +137,18 @@ dispatch_scatter_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n
   __shared__ int wc[kDispWarps][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispThreads + threadIdx.x;
+  // this token's experts, kept in registers
+  int ek[KMAX];
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k) ek[k] = (t < T && k < K) ? idx[t * K + k] : -1;
   uint32_t mask[NW];
-  token_mask<NW>(idx, t, T, K, mask);
+#pragma unroll
+  for (int w = 0; w < NW; ++w) mask[w] = 0;
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k)
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+      if (ek[k] >= 0 && (ek[k] >> 5) == w) mask[w] |= 1u << (ek[k] & 31);
   warp_counts<NW>(mask, n, warp, lane, wc);
   __syncthreads();
   for (int e = threadIdx.x; e < n; e += blockDim.x) {
@@ -151,13 +170,13 @@ dispatch_scatter_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n
       const unsigned bal = __ballot_sync(kFull, has);
       if (has) {
         const int pos = wc[warp][e] + __popc(bal & lt);
-        for (int k = 0; k < K; ++k) {
-          if (idx[t * K + k] == e) {
-            const int64_t slot = t * K + k;
-            perm[pos] = static_cast<int32_t>(slot);
-            inv[slot] = pos;
-          }
-        }
+        int kk = 0;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k)
+          if (ek[k] == e) kk = k;
+        const int64_t slot = t * K + kk;
+        perm[pos] = static_cast<int32_t>(slot);
+        inv[slot] = pos;
       }
     }
   }
@@ -185,7 +204,12 @@ gather_rows_kernel(const T* __restrict__ u, const int32_t* __restrict__ perm, in
 // ---------------------------------------------------------------------------
 // combine (eq. (9)): h_t = u_t + ysh_t + sum_k w[t,k] * y[inv[t*K+k]], in
 // fp32, in exactly this order (one fused multiply-add per k), rounded once.
+// One warp per token; the K expert rows of a column block are loaded in
+// batches of kCombineBatch before any of them is used, so their DRAM
+// latencies overlap instead of forming a chain.
 // ---------------------------------------------------------------------------
+constexpr int kCombineBatch = 8;
+
 template <typename T>
 __global__ void __launch_bounds__(256)
 combine_kernel(const T* __restrict__ u, const float* __restrict__ ysh, const T* __restrict__ y,
@@ -196,64 +220,43 @@ combine_kernel(const T* __restrict__ u, const float* __restrict__ ysh, const T* 
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        t < Tn; t += warps) {
-    // lane k < K holds row inv[t*K+k] and gate w[t*K+k]
-    int my_row = 0;
-    float my_w = 0.0f;
-    if (lane < K) {
-      my_row = inv[t * K + lane];
-      my_w = w[t * K + lane];
-    }
-    for (int c = lane * V; c < d; c += 32 * V) {
+    // lane k < K holds row inv[t*K+k] and gate w[t*K+k]; shuffles hand them out
+    const int my_row = lane < K ? inv[t * K + lane] : 0;
+    const float my_w = lane < K ? w[t * K + lane] : 0.0f;
+    // the trip count is the same for every lane, so the shuffles stay converged
+    for (int c0 = 0; c0 < d; c0 += 32 * V) {
+      const int c = c0 + lane * V;
+      const bool live = c < d;
       float acc[V], tmp[V];
-      Vec16<T>::load(u + t * d + c, acc);
+      if (live) {
+        Vec16<T>::load(u + t * d + c, acc);
 #pragma unroll
-      for (int i = 0; i < V; i += 4) {
-        Vec16<float>::load(ysh + t * d + c + i, tmp);
+        for (int i = 0; i < V; i += 4) {
+          Vec16<float>::load(ysh + t * d + c + i, tmp);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i + j] += tmp[j];
+          for (int j = 0; j < 4; ++j) acc[i + j] += tmp[j];
+        }
       }
-      for (int k = 0; k < K; ++k) {
-        const int64_t r = __shfl_sync(kFull, my_row, k);
-        const float wk = __shfl_sync(kFull, my_w, k);
-        Vec16<T>::load(y + r * d + c, tmp);
+      for (int k0 = 0; k0 < K; k0 += kCombineBatch) {
+        uint4 raw[kCombineBatch];
+        float wk[kCombineBatch];
 #pragma unroll
-        for (int j = 0; j < V; ++j) acc[j] = fmaf(wk, tmp[j], acc[j]);
+        for (int kk = 0; kk < kCombineBatch; ++kk) {
+          const int k = k0 + kk;
+          const int64_t r = __shfl_sync(kFull, my_row, k & 31);
+          wk[kk] = __shfl_sync(kFull, my_w, k & 31);
+          if (live && k < K) raw[kk] = *reinterpret_cast<const uint4*>(y + r * d + c);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kCombineBatch; ++kk) {
+          if (live && k0 + kk < K) {
+            Vec16<T>::load(reinterpret_cast<const T*>(&raw[kk]), tmp);
+#pragma unroll
+            for (int j = 0; j < V; ++j) acc[j] = fmaf(wk[kk], tmp[j], acc[j]);
+          }
+        }
       }
-      Vec16<T>::store(h + t * d + c, acc);
-    }
-  }
-}
-
-// The loop above keeps all lanes converged only while every lane runs the
-// same number of column iterations: d is a multiple of 32*V for that kernel.
-// Other widths use this one (each lane reads inv / w itself).
-template <typename T>
-__global__ void __launch_bounds__(256)
-combine_kernel_any(const T* __restrict__ u, const float* __restrict__ ysh, const T* __restrict__ y,
-                   const float* __restrict__ w, const int32_t* __restrict__ inv, int64_t Tn, int d,
-                   int K, T* __restrict__ h) {
-  constexpr int V = Vec16<T>::N;
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       t < Tn; t += warps) {
-    for (int c = lane * V; c < d; c += 32 * V) {
-      float acc[V], tmp[V];
-      Vec16<T>::load(u + t * d + c, acc);
-#pragma unroll
-      for (int i = 0; i < V; i += 4) {
-        Vec16<float>::load(ysh + t * d + c + i, tmp);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i + j] += tmp[j];
-      }
-      for (int k = 0; k < K; ++k) {
-        const int64_t r = inv[t * K + k];
-        const float wk = w[t * K + k];
-        Vec16<T>::load(y + r * d + c, tmp);
-#pragma unroll
-        for (int j = 0; j < V; ++j) acc[j] = fmaf(wk, tmp[j], acc[j]);
-      }
-      Vec16<T>::store(h + t * d + c, acc);
+      if (live) Vec16<T>::store(h + t * d + c, acc);
     }
   }
 }
@@ -455,8 +458,15 @@ int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_
   if (int rc = check_launch()) return rc;
 #define MOE_SCATTER_CASE(W)                                                                  \
   case W:                                                                                    \
-    dispatch_scatter_kernel<W><<<static_cast<unsigned>(nch), kDispThreads, 0, st>>>(           \
-        idx, T, K, n, chunk_base, perm, inv);                                                \
+    if (K <= 8)                                                                              \
+      dispatch_scatter_kernel<W, 8><<<static_cast<unsigned>(nch), kDispThreads, 0, st>>>(     \
+          idx, T, K, n, chunk_base, perm, inv);                                              \
+    else if (K <= 16)                                                                        \
+      dispatch_scatter_kernel<W, 16><<<static_cast<unsigned>(nch), kDispThreads, 0, st>>>(    \
+          idx, T, K, n, chunk_base, perm, inv);                                              \
+    else                                                                                     \
+      dispatch_scatter_kernel<W, 32><<<static_cast<unsigned>(nch), kDispThreads, 0, st>>>(    \
+          idx, T, K, n, chunk_base, perm, inv);                                              \
     break;
   switch (nw) {
     MOE_SCATTER_CASE(1) MOE_SCATTER_CASE(2) MOE_SCATTER_CASE(3) MOE_SCATTER_CASE(4)
@@ -486,21 +496,14 @@ int launch_combine(int dtype, const void* u, const float* ysh, const void* y, co
                    const int32_t* inv, int64_t T, int d, int K, void* h, cudaStream_t st) {
   if (T == 0) return MOE_OK;
   const unsigned grid = grid_for_rows(T, 8);
-  const int V = dtype == MOE_DTYPE_BF16 ? 8 : 4;
-  const bool uniform = (d % (32 * V)) == 0 && K <= 32;
-  if (dtype == MOE_DTYPE_BF16) {
-    auto* uu = static_cast<const bf16*>(u);
-    auto* yy = static_cast<const bf16*>(y);
-    auto* hh = static_cast<bf16*>(h);
-    if (uniform) combine_kernel<bf16><<<grid, 256, 0, st>>>(uu, ysh, yy, w, inv, T, d, K, hh);
-    else combine_kernel_any<bf16><<<grid, 256, 0, st>>>(uu, ysh, yy, w, inv, T, d, K, hh);
-  } else {
-    auto* uu = static_cast<const float*>(u);
-    auto* yy = static_cast<const float*>(y);
-    auto* hh = static_cast<float*>(h);
-    if (uniform) combine_kernel<float><<<grid, 256, 0, st>>>(uu, ysh, yy, w, inv, T, d, K, hh);
-    else combine_kernel_any<float><<<grid, 256, 0, st>>>(uu, ysh, yy, w, inv, T, d, K, hh);
-  }
+  if (dtype == MOE_DTYPE_BF16)
+    combine_kernel<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16*>(u), ysh,
+                                               static_cast<const bf16*>(y), w, inv, T, d, K,
+                                               static_cast<bf16*>(h));
+  else
+    combine_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(u), ysh,
+                                                static_cast<const float*>(y), w, inv, T, d, K,
+                                                static_cast<float*>(h));
   count_launch();
   return check_launch();
 }

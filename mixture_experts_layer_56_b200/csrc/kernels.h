@@ -6,7 +6,7 @@
 
 namespace moe {
 
-constexpr int kDispatchChunk = 256;  // tokens per dispatch block
+constexpr int kDispatchChunk = 128;  // tokens per dispatch block
 
 inline int64_t dispatch_num_chunks(int64_t T) { return (T + kDispatchChunk - 1) / kDispatchChunk; }
 int router_num_ctas(int64_t T);

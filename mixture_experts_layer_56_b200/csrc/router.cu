@@ -20,33 +20,64 @@ namespace {
 constexpr int kRouterWarps = 4;
 constexpr int kTokPerWarp = 8;
 constexpr int kTokPerCta = kRouterWarps * kTokPerWarp;  // 32
-constexpr int kChunk = 32;
 
-// Stage rows [r0, r0+nr) x columns [j0, j0+32) of a row-major [nrows, d]
-// matrix into dst[j][r] (fp32, zero outside the matrix).
+// Eight consecutive elements of a row as fp32 (zero outside the matrix).
 template <typename TIn>
-__device__ __forceinline__ void stage_transposed(const TIn* __restrict__ src, int64_t r0, int nr,
-                                                 int64_t nrows, int d, int j0, float* dst,
-                                                 int ld_dst) {
-  constexpr int V = Vec16<TIn>::N;      // elements per 16-byte load
-  constexpr int PER_ROW = kChunk / V;   // loads per row chunk
-  const bool vec_ok = (d % V) == 0;
-  for (int i = threadIdx.x; i < nr * PER_ROW; i += blockDim.x) {
-    const int rr = i / PER_ROW;
-    const int c = (i - rr * PER_ROW) * V;
-    const int64_t row = r0 + rr;
-    float v[V];
-    const int j = j0 + c;
-    if (row < nrows && vec_ok && j + V <= d) {
-      Vec16<TIn>::load(src + row * d + j, v);
+struct Row8;
+template <>
+struct Row8<bf16> {
+  uint4 raw;
+  __device__ __forceinline__ void load(const bf16* __restrict__ src, int64_t row, int64_t nrows,
+                                       int d, int j) {
+    if (row < nrows && j + 8 <= d) {
+      raw = *reinterpret_cast<const uint4*>(src + row * d + j);
     } else {
+      uint16_t h[8];
 #pragma unroll
-      for (int q = 0; q < V; ++q)
-        v[q] = (row < nrows && j + q < d) ? to_f32(src[row * d + j + q]) : 0.0f;
+      for (int q = 0; q < 8; ++q)
+        h[q] = (row < nrows && j + q < d)
+                   ? reinterpret_cast<const uint16_t*>(src)[row * d + j + q] : uint16_t(0);
+      raw = make_uint4(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16),
+                       h[4] | (uint32_t(h[5]) << 16), h[6] | (uint32_t(h[7]) << 16));
     }
-#pragma unroll
-    for (int q = 0; q < V; ++q) dst[(c + q) * ld_dst + rr] = v[q];
   }
+  __device__ __forceinline__ float get(int q) const {
+    const uint32_t w = q < 2 ? raw.x : q < 4 ? raw.y : q < 6 ? raw.z : raw.w;
+    return __uint_as_float((q & 1) ? (w & 0xffff0000u) : (w << 16));
+  }
+};
+template <>
+struct Row8<float> {
+  float4 lo, hi;
+  __device__ __forceinline__ void load(const float* __restrict__ src, int64_t row, int64_t nrows,
+                                       int d, int j) {
+    if (row < nrows && j + 8 <= d && (d & 3) == 0) {
+      lo = *reinterpret_cast<const float4*>(src + row * d + j);
+      hi = *reinterpret_cast<const float4*>(src + row * d + j + 4);
+    } else {
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = (row < nrows && j + q < d) ? src[row * d + j + q] : 0.0f;
+      lo = make_float4(v[0], v[1], v[2], v[3]);
+      hi = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  }
+  __device__ __forceinline__ float get(int q) const {
+    const float4& v = q < 4 ? lo : hi;
+    const int r = q & 3;
+    return r == 0 ? v.x : r == 1 ? v.y : r == 2 ? v.z : v.w;
+  }
+};
+
+// d-chunk staged per step: as long as shared memory allows (the global loads
+// of the next chunk are in flight while the current one is multiplied).
+template <int EPT>
+constexpr int router_chunk() {
+  return EPT <= 2 ? 128 : (EPT <= 4 ? 64 : 32);
+}
+template <int EPT>
+constexpr int router_smem_bytes() {
+  return router_chunk<EPT>() * (kTokPerCta + EPT * 32) * 4;
 }
 
 template <typename TIn, int EPT, bool STATS>
@@ -55,12 +86,38 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
                    const float* __restrict__ bias, int64_t T, int d, int n, int K, int flags,
                    int32_t* __restrict__ idx, float* __restrict__ w, float* __restrict__ pstat) {
   constexpr int NP = EPT * 32;
-  __shared__ __align__(16) float sU[kChunk][kTokPerCta];
-  __shared__ __align__(16) float sE[kChunk][NP];
+  constexpr int KC = router_chunk<EPT>();
+  constexpr int NT = kRouterWarps * 32;      // threads
+  constexpr int UG = KC / 8 * kTokPerCta / NT;  // u items (8 columns each) per thread
+  constexpr int EG = KC / 8 * NP / NT;          // E items per thread
+  // one d-chunk of u (tokens) and E (experts), transposed to [j][row], fp32
+  extern __shared__ __align__(16) float smem_f[];
+  float (*sU)[kTokPerCta] = reinterpret_cast<float (*)[kTokPerCta]>(smem_f);
+  float (*sE)[NP] = reinterpret_cast<float (*)[NP]>(smem_f + KC * kTokPerCta);
 
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTokPerCta;
+
+  // staging assignment: item i = tid + NT*k covers 8 columns of one row,
+  // row = i % rows, column group = i / rows.  Within a warp the group is
+  // fixed and the rows are consecutive, so the transposed stores hit 32
+  // distinct banks.
+  Row8<TIn> pu[UG];
+  Row8<TIn> pe[EG];
+  auto prefetch = [&](int j0) {
+#pragma unroll
+    for (int k = 0; k < UG; ++k) {
+      const int i = tid + NT * k;
+      pu[k].load(u, t0 + i % kTokPerCta, T, d, j0 + (i / kTokPerCta) * 8);
+    }
+#pragma unroll
+    for (int k = 0; k < EG; ++k) {
+      const int i = tid + NT * k;
+      pe[k].load(E, i % NP, n, d, j0 + (i / NP) * 8);
+    }
+  };
 
   float acc[kTokPerWarp][EPT];
 #pragma unroll
@@ -68,12 +125,26 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
 #pragma unroll
     for (int q = 0; q < EPT; ++q) acc[i][q] = 0.0f;
 
-  for (int j0 = 0; j0 < d; j0 += kChunk) {
-    stage_transposed<TIn>(u, t0, kTokPerCta, T, d, j0, &sU[0][0], kTokPerCta);
-    stage_transposed<TIn>(E, 0, NP, n, d, j0, &sE[0][0], NP);
+  prefetch(0);
+  for (int j0 = 0; j0 < d; j0 += KC) {
+    __syncthreads();  // the previous chunk's reads are done
+#pragma unroll
+    for (int k = 0; k < UG; ++k) {
+      const int i = tid + NT * k;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) sU[(i / kTokPerCta) * 8 + q][i % kTokPerCta] = pu[k].get(q);
+    }
+#pragma unroll
+    for (int k = 0; k < EG; ++k) {
+      const int i = tid + NT * k;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) sE[(i / NP) * 8 + q][i % NP] = pe[k].get(q);
+    }
     __syncthreads();
-#pragma unroll 4
-    for (int j = 0; j < kChunk; ++j) {
+    if (j0 + KC < d) prefetch(j0 + KC);  // in flight during the FMAs below
+    const int jn = min(KC, d - j0);
+#pragma unroll 8
+    for (int j = 0; j < jn; ++j) {
       float ev[EPT];
 #pragma unroll
       for (int q = 0; q < EPT; ++q) ev[q] = sE[j][lane + 32 * q];
@@ -85,7 +156,6 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
 #pragma unroll
         for (int q = 0; q < EPT; ++q) acc[i][q] = fmaf(uv[i], ev[q], acc[i][q]);
     }
-    __syncthreads();
   }
 
   float b[EPT];
@@ -188,11 +258,16 @@ int launch_router_t(const TIn* u, const TIn* E, const float* bias, int64_t T, in
   const int ept = (n + 31) / 32;
   const unsigned grid = static_cast<unsigned>((T + kTokPerCta - 1) / kTokPerCta);
   const dim3 block(kRouterWarps * 32);
-#define MOE_ROUTER_CASE(N)                                                                \
-  case N:                                                                                 \
-    router_topk_kernel<TIn, N, STATS><<<grid, block, 0, st>>>(u, E, bias, T, d, n, K, flags, \
-                                                               idx, w, pstat);            \
-    break;
+#define MOE_ROUTER_CASE(N)                                                                  \
+  case N: {                                                                                 \
+    auto kern = router_topk_kernel<TIn, N, STATS>;                                          \
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,             \
+                             router_smem_bytes<N>()) != cudaSuccess)                        \
+      return MOE_ERR_CUDA;                                                                  \
+    kern<<<grid, block, router_smem_bytes<N>(), st>>>(u, E, bias, T, d, n, K, flags, idx, w, \
+                                                     pstat);                                \
+    break;                                                                                  \
+  }
   switch (ept) {
     MOE_ROUTER_CASE(1)
     MOE_ROUTER_CASE(2)
