@@ -252,7 +252,8 @@ def run_ours(args):
 
     wl = S.WORKLOADS[args.config]
     x = S.make_inputs(wl)
-    layer = MoELayer(x, dev, host_io=True)
+    flags = {"auto": 0, "single": L.MOE_FLAG_GEMM_SINGLE_CTA, "pair": L.MOE_FLAG_GEMM_CTA_PAIR}[args.gemm]
+    layer = MoELayer(x, dev, flags=flags, host_io=True)
     u = to_device(x.u, dev)
     h = torch.empty_like(u)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -363,6 +364,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic",
             "config": {"workload": workload_desc(wl), "tokens_per_gpu_step": wl.T,
+                       "gemm_tiles": args.gemm,
                        "parallelism": f"replicas x{world} (token batches, no collective)",
                        "l2": "flushed between steps (256 MB memset outside the step events)",
                        "init": "seeded splitmix64/Box-Muller normals, bf16"},
@@ -408,6 +410,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm", default="auto", choices=["auto", "single", "pair"],
+                    help="tile shape of the expert GEMMs (default: chosen by the library)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

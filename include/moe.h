@@ -72,6 +72,13 @@ enum {
      csdn.net DeepSeekMoE article describes in words, §2.3).  Default (0):
      the bias is part of the logit for both selection and softmax. */
   MOE_FLAG_BIAS_SELECT_ONLY = 1,
+  /* Tile shape of the bf16 expert GEMMs (default: chosen from the average
+     rows per routed expert).  SINGLE_CTA: 128-row tiles, one SM each.
+     CTA_PAIR: 256-row tiles computed by the two SMs of a 2-CTA cluster
+     (tcgen05 cta_group::2).  Setting both is MOE_ERR_SHAPE.  Results are the
+     same up to fp32 summation order inside the tensor cores. */
+  MOE_FLAG_GEMM_SINGLE_CTA = 2,
+  MOE_FLAG_GEMM_CTA_PAIR = 4,
 };
 
 /* Layer shape.  Limits: 1 <= n_routed <= 256, 1 <= top_k <= min(n_routed, 32),

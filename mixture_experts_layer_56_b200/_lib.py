@@ -17,6 +17,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 MOE_DTYPE_F32 = 0
 MOE_DTYPE_BF16 = 1
 MOE_FLAG_BIAS_SELECT_ONLY = 1
+MOE_FLAG_GEMM_SINGLE_CTA = 2
+MOE_FLAG_GEMM_CTA_PAIR = 4
 
 MOE_OK = 0
 MOE_ERR_NULLPTR = -1

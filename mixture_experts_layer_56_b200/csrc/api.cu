@@ -130,7 +130,10 @@ int validate(const moe_shape_t* s) {
       s->top_k > s->n_routed || s->top_k > 32 || s->n_shared < 0 || s->n_shared > 64 ||
       s->inter < 1)
     return MOE_ERR_SHAPE;
-  if ((s->flags & ~MOE_FLAG_BIAS_SELECT_ONLY) != 0) return MOE_ERR_SHAPE;
+  const int32_t known = MOE_FLAG_BIAS_SELECT_ONLY | MOE_FLAG_GEMM_SINGLE_CTA | MOE_FLAG_GEMM_CTA_PAIR;
+  if ((s->flags & ~known) != 0) return MOE_ERR_SHAPE;
+  if ((s->flags & MOE_FLAG_GEMM_SINGLE_CTA) && (s->flags & MOE_FLAG_GEMM_CTA_PAIR))
+    return MOE_ERR_SHAPE;
   // positions are int32; rows address TMA coordinates (int32)
   if (s->T * static_cast<int64_t>(s->top_k) > 0x7fffffffLL) return MOE_ERR_SHAPE;
   if (s->inter % 64 != 0) return MOE_ERR_SHAPE;
@@ -175,9 +178,13 @@ T* at(void* ws, size_t off) {
 }
 
 // expert FFNs on workspace-resident gathered rows
+// y_slot_order: write routed expert outputs at row perm[p] (token slot
+// t*K+k) instead of row p, so that the combine reads each token's rows
+// contiguously.
 int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const int32_t* perm,
                    const int32_t* offsets, const void* W13, const void* W2, const void* W13_s,
-                   const void* W2_s, void* y, float* ysh, void* ws, cudaStream_t st, int sms) {
+                   const void* W2_s, void* y, float* ysh, void* ws, cudaStream_t st, int sms,
+                   bool y_slot_order) {
   const int64_t T = s.T, K = s.top_k, rows = T * K;
   const int d = s.d, I = s.inter, n = s.n_routed, ns = s.n_shared;
   void* xperm = at<void>(ws, L.xperm);
@@ -206,20 +213,36 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
 
   using namespace sm100;
   const uint64_t d64 = static_cast<uint64_t>(d), I64 = static_cast<uint64_t>(I);
-  const int64_t routed_mt_ub = (rows + 127) / 128 + (rows < n ? rows : n);
-  const int64_t shared_mt = ns > 0 ? (T + 127) / 128 : 0;
   int32_t* status = at<int32_t>(ws, L.status);
+  // 256-row tiles on CTA pairs once experts average at least half such a
+  // tile; 128-row tiles on single SMs otherwise (decode-sized batches)
+  bool pair = rows >= static_cast<int64_t>(n) * 128;
+  if (s.flags & MOE_FLAG_GEMM_SINGLE_CTA) pair = false;
+  if (s.flags & MOE_FLAG_GEMM_CTA_PAIR) pair = true;
+  const int BM = pair ? 256 : 128;
+  const int64_t routed_mt_ub = (rows + BM - 1) / BM + (rows < n ? rows : n);
+  const int64_t shared_mt = ns > 0 ? (T + BM - 1) / BM : 0;
+  auto launch = [&](int BN, int epi, const GemmMaps& m, const GroupedGemmArgs& a) {
+    const int64_t tiles = routed_mt_ub * a.nt_routed + shared_mt * a.nt_shared;
+    if (pair) {
+      const int64_t cl = tiles < sms / 2 ? tiles : sms / 2;
+      return launch_grouped_gemm_pair(BN, epi, m, a, static_cast<int>(cl), st);
+    }
+    const int64_t grid = tiles < sms ? tiles : sms;
+    return launch_grouped_gemm(BN, epi, m, a, static_cast<int>(grid), st);
+  };
 
   // ---- gate/up + SwiGLU ---------------------------------------------------
   {
     const int BN = (2 * I) % 256 == 0 ? 256 : 128;
+    const uint32_t bbox = pair ? BN / 2 : BN;
     GemmMaps m;
     bool ok = make_map_bf16(&m.a_r, 2, xperm, d64, rows, 1, d64 * 2, 0, 128) &&
-              make_map_bf16(&m.b_r, 3, W13, d64, 2 * I64, n, d64 * 2, 2 * I64 * d64 * 2, BN);
+              make_map_bf16(&m.b_r, 3, W13, d64, 2 * I64, n, d64 * 2, 2 * I64 * d64 * 2, bbox);
     if (ns > 0) {
       ok = ok && make_map_bf16(&m.a_s, 2, u, d64, T, 1, d64 * 2, 0, 128) &&
            make_map_bf16(&m.b_s, 3, W13_s, d64, 2 * I64 * ns, 1, d64 * 2, 2 * I64 * ns * d64 * 2,
-                         BN);
+                         bbox);
     } else {
       m.a_s = m.a_r;
       m.b_s = m.b_r;
@@ -239,20 +262,19 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     a.out_s = act_s;
     a.ld_s = static_cast<int64_t>(I) * ns;
     a.status = status;
-    const int64_t tiles = routed_mt_ub * a.nt_routed + shared_mt * a.nt_shared;
-    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
     Stage sg(MOE_KERNEL_GEMM_GATE_UP, st);
-    if (int rc = launch_grouped_gemm(BN, kEpiSwiGLU, m, a, grid, st)) return rc;
+    if (int rc = launch(BN, kEpiSwiGLU, m, a)) return rc;
   }
   // ---- down projection ----------------------------------------------------
   {
     const int BN = d % 256 == 0 ? 256 : (d % 128 == 0 ? 128 : 64);
+    const uint32_t bbox = pair ? BN / 2 : BN;
     GemmMaps m;
     bool ok = make_map_bf16(&m.a_r, 2, act, I64, rows, 1, I64 * 2, 0, 128) &&
-              make_map_bf16(&m.b_r, 3, W2, I64, d64, n, I64 * 2, d64 * I64 * 2, BN);
+              make_map_bf16(&m.b_r, 3, W2, I64, d64, n, I64 * 2, d64 * I64 * 2, bbox);
     if (ns > 0) {
       ok = ok && make_map_bf16(&m.a_s, 2, act_s, I64 * ns, T, 1, I64 * ns * 2, 0, 128) &&
-           make_map_bf16(&m.b_s, 3, W2_s, I64, d64, ns, I64 * 2, d64 * I64 * 2, BN);
+           make_map_bf16(&m.b_s, 3, W2_s, I64, d64, ns, I64 * 2, d64 * I64 * 2, bbox);
     } else {
       m.a_s = m.a_r;
       m.b_s = m.b_r;
@@ -269,13 +291,12 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     a.nt_shared = d / BN;
     a.out_r = y;
     a.ld_r = d;
+    a.row_map_r = y_slot_order ? perm : nullptr;
     a.out_s = ysh;
     a.ld_s = d;
     a.status = status;
-    const int64_t tiles = routed_mt_ub * a.nt_routed + shared_mt * a.nt_shared;
-    const int grid = static_cast<int>(tiles < sms ? tiles : sms);
     Stage sg(MOE_KERNEL_GEMM_DOWN, st);
-    if (int rc = launch_grouped_gemm(BN, kEpiPlain, m, a, grid, st)) return rc;
+    if (int rc = launch(BN, kEpiPlain, m, a)) return rc;
   }
   return MOE_OK;
 }
@@ -304,10 +325,14 @@ int forward_device(const moe_shape_t& s, const Layout& L, const void* u, const v
                                  at<int32_t>(ws, L.chunk_base), counts, offsets, perm, inv, st))
       return rc;
   }
-  if (int rc = run_expert_ffn(s, L, u, perm, offsets, W13, W2, W13_s, W2_s, y, ysh, ws, st, sms))
+  // the tensor-core path writes y in token-slot order (the combine then
+  // reads each token's rows contiguously); the fp32 path keeps expert order
+  const bool slot_order = s.dtype == MOE_DTYPE_BF16;
+  if (int rc = run_expert_ffn(s, L, u, perm, offsets, W13, W2, W13_s, W2_s, y, ysh, ws, st, sms,
+                              slot_order))
     return rc;
   Stage sg(MOE_KERNEL_COMBINE, st);
-  return launch_combine(s.dtype, u, ysh, y, w, inv, T, s.d, K, h, st);
+  return launch_combine(s.dtype, u, ysh, y, w, slot_order ? nullptr : inv, T, s.d, K, h, st);
 }
 
 bool shared_ptrs_ok(const moe_shape_t& s, const void* W13_s, const void* W2_s) {
@@ -464,7 +489,7 @@ int moe_expert_ffn(const moe_shape_t* shape, const void* u, const int32_t* perm,
   DeviceInfo di;
   if (int rc = device_info(&di)) return rc;
   return run_expert_ffn(*shape, L, u, perm, offsets, W13, W2, W13_s, W2_s, y, ysh, ws,
-                        static_cast<cudaStream_t>(stream), di.sms);
+                        static_cast<cudaStream_t>(stream), di.sms, /*y_slot_order=*/false);
 }
 
 int moe_combine(const moe_shape_t* shape, const void* u, const float* ysh, const void* y,

@@ -53,6 +53,19 @@ template <> struct Vec16<float> {
   }
 };
 
+// SiLU(g) * u = g * u / (1 + e^-g).  e^-g is computed as 2^(-g log2 e) and
+// the reciprocal directly, both on the special-function unit (ex2.approx,
+// rcp.approx: a few ulp each, far below the bf16 rounding that follows).
+// g is clamped at -80 so that 1 + e^-g stays finite (the product is then 0
+// to within 1e-33).
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  const float gc = fmaxf(g, -80.0f);
+  float e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(gc * -1.4426950408889634f));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+  return g * r * u;
+}
+
 // The workspace begins with a 256-byte header whose first int32 is the
 // status word that kernels set when a bounded wait gives up.
 __device__ __forceinline__ void record_status(int32_t* status, int32_t code) {

@@ -33,7 +33,7 @@ namespace sm100 {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // 4 role warps + 8 epilogue warps
 constexpr int kMaxGroups = 257;  // 256 routed + 1 shared
 
 template <int BN> struct Cfg;
@@ -115,7 +115,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 128);
+      mbar_init(tempty_bar(a), 8);  // one arrive per epilogue warp
     }
     mbar_init(drain_bar, 1);
     abort_flag = 0;
@@ -249,7 +249,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------- epilogue -----
-    const int q = warp & 3;
+    const int q = warp & 3;          // TMEM lane quarter of this warp
+    const int hcol = (warp - 4) >> 2;  // which half of the tile's columns it drains
     const int r = q * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
@@ -261,6 +262,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
       const int rows_valid = grp_rows[ti.g] - ti.m_blk * BM;
       const int64_t orow = static_cast<int64_t>(grp_row0[ti.g]) + ti.m_blk * BM + r;
       const bool live = r < rows_valid;
+      // routed rows of the plain epilogue may be remapped (token-slot order)
+      const int64_t prow = (EPI == kEpiPlain && !ti.shared && args.row_map_r != nullptr && live)
+                               ? static_cast<int64_t>(args.row_map_r[orow])
+                               : orow;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
       if (EPI == kEpiSwiGLU) {
@@ -268,7 +273,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
         const int64_t ld = ti.shared ? args.ld_s : args.ld_r;
         const int64_t col0 = static_cast<int64_t>(ti.n_blk) * (BN / 2);
 #pragma unroll 1
-        for (int c = 0; c < BN / 64; ++c) {
+        for (int c = hcol * (BN / 128); c < (hcol + 1) * (BN / 128); ++c) {
           const int pair = c >> 1, half = c & 1;
           const int gcol = pair * 128 + half * 32;
           float gv[32], uv[32];
@@ -281,17 +286,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
             for (int v = 0; v < 4; ++v) {
               float o[8];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float x = gv[v * 8 + j];
-                o[j] = x / (1.0f + __expf(-x)) * uv[v * 8 + j];
-              }
+              for (int j = 0; j < 8; ++j) o[j] = silu_mul(gv[v * 8 + j], uv[v * 8 + j]);
               Vec16<bf16>::store(dst + v * 8, o);
             }
           }
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = hcol * (BN / 64); c < (hcol + 1) * (BN / 64); ++c) {
           float x[32];
           tmem_ld32(taddr + c * 32, x);
           tmem_ld_wait();
@@ -302,7 +304,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
 #pragma unroll
               for (int v = 0; v < 8; ++v) Vec16<float>::store(dst + v * 4, x + v * 4);
             } else {
-              bf16* dst = static_cast<bf16*>(args.out_r) + orow * args.ld_r + col;
+              bf16* dst = static_cast<bf16*>(args.out_r) + prow * args.ld_r + col;
 #pragma unroll
               for (int v = 0; v < 4; ++v) Vec16<bf16>::store(dst + v * 8, x + v * 8);
             }
@@ -310,7 +312,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
         }
       }
       tc_fence_before();
-      mbar_arrive(tempty_bar(acc));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
     }
   }
 

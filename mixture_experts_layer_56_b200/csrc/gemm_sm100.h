@@ -23,6 +23,7 @@ struct GroupedGemmArgs {
   int32_t nt_shared;       // BN-wide N tiles of the shared group
   void* out_r;             // routed output (bf16), row stride ld_r elements
   int64_t ld_r;
+  const int32_t* row_map_r;  // routed output row of position p: row_map_r[p] (NULL: p)
   void* out_s;             // shared output: bf16 (SwiGLU) or fp32 (plain)
   int64_t ld_s;
   int32_t* status;         // workspace status word
@@ -40,6 +41,11 @@ bool make_map_bf16(CUtensorMap* map, int rank, const void* base, uint64_t inner,
 
 int launch_grouped_gemm(int BN, int epi, const GemmMaps& maps, const GroupedGemmArgs& args,
                         int grid, cudaStream_t stream);
+
+// The same GEMM on 2-CTA clusters with 256-row tiles (gemm_sm100_pair.cu).
+// B maps must have box rows BN / 2.  `clusters` CTA pairs are launched.
+int launch_grouped_gemm_pair(int BN, int epi, const GemmMaps& maps, const GroupedGemmArgs& args,
+                             int clusters, cudaStream_t stream);
 
 }  // namespace sm100
 }  // namespace moe

@@ -1,0 +1,368 @@
+// Grouped expert GEMM on CTA pairs (tcgen05 cta_group::2): the same
+// computation as gemm_sm100.cu (gate/up + SwiGLU, or down projection, over
+// the shared group and the routed experts of the DeepSeekMoE layer, §3.2
+// eq. (9)) with 256-row tiles split over the two SMs of a cluster.
+//
+// The leader CTA (rank 0) issues every MMA of the pair: M = 256 (rows 0..127
+// from its own shared memory, 128..255 from the peer's), N = BN (B rows
+// split in halves the same way), accumulating 128 rows x BN fp32 columns in
+// each CTA's TMEM.  Each CTA loads its own A rows and B half with TMA; all
+// transaction bytes land on the leader's "full" barrier, whose expected
+// count the leader sets for both.  The leader's commits arrive on the
+// "empty" and "accumulator full" barriers of both CTAs at once; both
+// epilogues release an accumulator on the leader's "accumulator empty"
+// barrier.  Per CTA and k-block this moves 16 KB of A and BN*64 B of B,
+// against 16 KB + BN*128 B for one CTA computing half the tile alone.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "gemm_sm100.h"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace sm100 {
+
+namespace {
+
+constexpr int PBM = 256;   // rows per pair tile
+constexpr int HBM_ROWS = 128;  // rows per CTA
+constexpr int PBK = 64;
+constexpr int kPairThreads = 384;  // 4 role warps + 8 epilogue warps
+constexpr int kPairMaxGroups = 257;
+
+template <int BN> struct PairCfg;
+template <> struct PairCfg<256> { static constexpr int STAGES = 6; };
+template <> struct PairCfg<128> { static constexpr int STAGES = 8; };
+template <> struct PairCfg<64>  { static constexpr int STAGES = 9; };
+
+template <int BN>
+constexpr int pair_smem_bytes() {
+  return PairCfg<BN>::STAGES * (HBM_ROWS * PBK * 2 + (BN / 2) * PBK * 2) + 1024;
+}
+
+struct PairTile {
+  int g, shared, m_blk, n_blk;
+};
+
+__device__ __forceinline__ PairTile decode_pair_tile(int tile, const int32_t* tile_start, int G,
+                                                     int hs, int nt_r, int nt_s) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  PairTile t;
+  t.g = lo;
+  t.shared = (hs && lo == 0) ? 1 : 0;
+  const int nt = t.shared ? nt_s : nt_r;
+  const int local = tile - tile_start[lo];
+  t.m_blk = local / nt;
+  t.n_blk = local - t.m_blk * nt;
+  return t;
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kPairThreads, 1)
+grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
+                         const __grid_constant__ CUtensorMap tmA_s,
+                         const __grid_constant__ CUtensorMap tmB_r,
+                         const __grid_constant__ CUtensorMap tmB_s, const GroupedGemmArgs args) {
+  constexpr int STAGES = PairCfg<BN>::STAGES;
+  constexpr uint32_t A_BYTES = HBM_ROWS * PBK * 2;
+  constexpr uint32_t B_BYTES = (BN / 2) * PBK * 2;
+  constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t TMEM_COLS = 2 * BN;
+  constexpr uint32_t IDESC = idesc_bf16_f32(PBM, BN);
+  constexpr uint16_t kBoth = 0x3;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[2 * STAGES + 5];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  __shared__ int32_t tile_start[kPairMaxGroups + 1];
+  __shared__ int32_t grp_row0[kPairMaxGroups];
+  __shared__ int32_t grp_rows[kPairMaxGroups];
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t smem_base = smem_addr(smem);
+  const uint32_t bar_base = smem_addr(bars);
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = static_cast<int>(cluster_id_x());
+  const int nclusters = static_cast<int>(num_clusters_x());
+  const int hs = args.shared_rows > 0 ? 1 : 0;
+  const int G = args.n_routed + hs;
+  volatile int* abort_p = &abort_flag;
+
+  // ---- setup --------------------------------------------------------------
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);   // the leader's arrive (+ both CTAs' bytes)
+      mbar_init(empty_bar(s), 1);  // one multicast commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);   // one multicast commit
+      mbar_init(tempty_bar(a), 16);  // 8 epilogue warps x 2 CTAs (leader's copy)
+    }
+    mbar_init(drain_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    fence_async_shared();
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(smem_addr(&tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  for (int g = tid; g < G; g += kPairThreads) {
+    int rows, row0, nt;
+    if (hs && g == 0) {
+      rows = args.shared_rows; row0 = 0; nt = args.nt_shared;
+    } else {
+      const int e = g - hs;
+      row0 = args.offsets[e];
+      rows = args.offsets[e + 1] - row0;
+      nt = args.nt_routed;
+    }
+    grp_row0[g] = row0;
+    grp_rows[g] = rows;
+    tile_start[g + 1] = ((rows + PBM - 1) / PBM) * nt;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    const int beg = min(lane * per, G);
+    const int end = min(beg + per, G);
+    int sum = 0;
+    for (int i = beg; i < end; ++i) sum += tile_start[i + 1];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+    for (int i = beg; i < end; ++i) {
+      run += tile_start[i + 1];
+      tile_start[i + 1] = run;
+    }
+    if (lane == 0) tile_start[0] = 0;
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barrier inits and TMEM allocations visible to the pair
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  const int total_tiles = tile_start[G];
+
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer ----
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA_r);
+      tma_prefetch_desc(&tmB_r);
+      if (hs) {
+        tma_prefetch_desc(&tmA_s);
+        tma_prefetch_desc(&tmB_s);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < total_tiles && ok; tile += nclusters) {
+        const PairTile ti =
+            decode_pair_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+        const CUtensorMap* ma = ti.shared ? &tmA_s : &tmA_r;
+        const CUtensorMap* mb = ti.shared ? &tmB_s : &tmB_r;
+        const int row = grp_row0[ti.g] + ti.m_blk * PBM + static_cast<int>(rank) * HBM_ROWS;
+        const int nrow = ti.n_blk * BN + static_cast<int>(rank) * (BN / 2);
+        const int nkb = ti.shared ? args.kb_shared : args.kb_routed;
+        const int zbase = ti.shared ? 0 : ti.g - hs;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_p, args.status)) { ok = false; break; }
+          const uint32_t sa = smem_base + stage * STAGE_BYTES;
+          const uint32_t fb = leader ? full_bar(stage) : map_to_cta(full_bar(stage), 0);
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          tma_load_2d_pair(sa, ma, fb, kb * PBK, row);
+          tma_load_3d_pair(sa + A_BYTES, mb, fb, (kb % args.kb_per_expert) * PBK, nrow,
+                           zbase + kb / args.kb_per_expert);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ----------------------------------------- MMA issuer (leader only) ----
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < total_tiles && ok; tile += nclusters, ++it) {
+        const PairTile ti =
+            decode_pair_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+        const int nkb = ti.shared ? args.kb_shared : args.kb_routed;
+        const int acc = it & 1;
+        const uint32_t ap = (it >> 1) & 1;
+        if (!wait_bounded(tempty_bar(acc), ap ^ 1u, abort_p, args.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_bounded(full_bar(stage), phase, abort_p, args.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_base + stage * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < PBK / 16; ++k) {
+            mma_bf16_pair(d_tmem, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32),
+                          IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(empty_bar(stage), kBoth);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) mma_commit_pair(tfull_bar(acc), kBoth);
+      }
+      if (!ok) {
+        // wait for every MMA already issued before TMEM is released
+        mma_commit_pair(drain_bar, 0x1);
+        int dummy = 0;
+        wait_bounded(drain_bar, 0, &dummy, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------- epilogue -----
+    const int q = warp & 3;          // TMEM lane quarter of this warp
+    const int hcol = (warp - 4) >> 2;  // which half of the tile's columns it drains
+    const int r = q * 32 + lane;
+    const uint32_t tempty_leader0 = map_to_cta(tempty_bar(0), 0);
+    const uint32_t tempty_leader1 = map_to_cta(tempty_bar(1), 0);
+    int it = 0;
+    for (int tile = cluster; tile < total_tiles; tile += nclusters, ++it) {
+      const PairTile ti =
+          decode_pair_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+      const int acc = it & 1;
+      const uint32_t ap = (it >> 1) & 1;
+      if (!wait_bounded(tfull_bar(acc), ap, abort_p, args.status)) break;
+      tc_fence_after();
+      const int my0 = ti.m_blk * PBM + static_cast<int>(rank) * HBM_ROWS;
+      const int rows_valid = grp_rows[ti.g] - my0;
+      const int64_t orow = static_cast<int64_t>(grp_row0[ti.g]) + my0 + r;
+      const bool live = r < rows_valid;
+      // routed rows of the plain epilogue may be remapped (token-slot order)
+      const int64_t prow = (EPI == kEpiPlain && !ti.shared && args.row_map_r != nullptr && live)
+                               ? static_cast<int64_t>(args.row_map_r[orow])
+                               : orow;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+      if (EPI == kEpiSwiGLU) {
+        bf16* out = static_cast<bf16*>(ti.shared ? args.out_s : args.out_r);
+        const int64_t ld = ti.shared ? args.ld_s : args.ld_r;
+        const int64_t col0 = static_cast<int64_t>(ti.n_blk) * (BN / 2);
+#pragma unroll 1
+        for (int c = hcol * (BN / 128); c < (hcol + 1) * (BN / 128); ++c) {
+          const int pair = c >> 1, half = c & 1;
+          const int gcol = pair * 128 + half * 32;
+          float gv[32], uv[32];
+          tmem_ld32(taddr + gcol, gv);
+          tmem_ld32(taddr + gcol + 64, uv);
+          tmem_ld_wait();
+          if (live) {
+            bf16* dst = out + orow * ld + col0 + pair * 64 + half * 32;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              float o[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) o[j] = silu_mul(gv[v * 8 + j], uv[v * 8 + j]);
+              Vec16<bf16>::store(dst + v * 8, o);
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = hcol * (BN / 64); c < (hcol + 1) * (BN / 64); ++c) {
+          float x[32];
+          tmem_ld32(taddr + c * 32, x);
+          tmem_ld_wait();
+          if (live) {
+            const int64_t col = static_cast<int64_t>(ti.n_blk) * BN + c * 32;
+            if (ti.shared) {
+              float* dst = static_cast<float*>(args.out_s) + orow * args.ld_s + col;
+#pragma unroll
+              for (int v = 0; v < 8; ++v) Vec16<float>::store(dst + v * 4, x + v * 4);
+            } else {
+              bf16* dst = static_cast<bf16*>(args.out_r) + prow * args.ld_r + col;
+#pragma unroll
+              for (int v = 0; v < 4; ++v) Vec16<bf16>::store(dst + v * 8, x + v * 8);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // no CTA of the pair leaves while the other still works
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+template <int BN, int EPI>
+int launch_pair_impl(const GemmMaps& m, const GroupedGemmArgs& args, int clusters,
+                     cudaStream_t stream) {
+  static bool attr_done = false;
+  auto kern = grouped_gemm_pair_kernel<BN, EPI>;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pair_smem_bytes<BN>()) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    attr_done = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
+  cfg.dynamicSmemBytes = pair_smem_bytes<BN>();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, m.a_r, m.a_s, m.b_r, m.b_s, args) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  count_launch();
+  return check_launch();
+}
+
+}  // namespace
+
+int launch_grouped_gemm_pair(int BN, int epi, const GemmMaps& maps, const GroupedGemmArgs& args,
+                             int clusters, cudaStream_t stream) {
+  if (clusters <= 0) return MOE_OK;
+  if (epi == kEpiSwiGLU) {
+    if (BN == 256) return launch_pair_impl<256, kEpiSwiGLU>(maps, args, clusters, stream);
+    if (BN == 128) return launch_pair_impl<128, kEpiSwiGLU>(maps, args, clusters, stream);
+  } else {
+    if (BN == 256) return launch_pair_impl<256, kEpiPlain>(maps, args, clusters, stream);
+    if (BN == 128) return launch_pair_impl<128, kEpiPlain>(maps, args, clusters, stream);
+    if (BN == 64) return launch_pair_impl<64, kEpiPlain>(maps, args, clusters, stream);
+  }
+  return MOE_ERR_SHAPE;
+}
+
+}  // namespace sm100
+}  // namespace moe

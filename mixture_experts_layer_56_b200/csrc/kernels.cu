@@ -190,14 +190,24 @@ __global__ void __launch_bounds__(256)
 gather_rows_kernel(const T* __restrict__ u, const int32_t* __restrict__ perm, int64_t rows, int d,
                    int K, T* __restrict__ xperm) {
   constexpr int V = Vec16<T>::N;
+  constexpr int U = 4;  // 16-byte loads in flight per lane before the stores
   const int lane = threadIdx.x & 31;
+  const int nv = d / V;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t p = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        p < rows; p += warps) {
     const int64_t t = perm[p] / K;
     const uint4* src = reinterpret_cast<const uint4*>(u + t * d);
     uint4* dst = reinterpret_cast<uint4*>(xperm + p * d);
-    for (int c = lane; c < d / V; c += 32) dst[c] = src[c];
+    for (int c0 = lane; c0 < nv; c0 += 32 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k)
+        if (c0 + 32 * k < nv) v[k] = src[c0 + 32 * k];
+#pragma unroll
+      for (int k = 0; k < U; ++k)
+        if (c0 + 32 * k < nv) dst[c0 + 32 * k] = v[k];
+    }
   }
 }
 
@@ -208,10 +218,10 @@ gather_rows_kernel(const T* __restrict__ u, const int32_t* __restrict__ perm, in
 // batches of kCombineBatch before any of them is used, so their DRAM
 // latencies overlap instead of forming a chain.
 // ---------------------------------------------------------------------------
-constexpr int kCombineBatch = 8;
+constexpr int kCombineBatch = 4;
 
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 combine_kernel(const T* __restrict__ u, const float* __restrict__ ysh, const T* __restrict__ y,
                const float* __restrict__ w, const int32_t* __restrict__ inv, int64_t Tn, int d,
                int K, T* __restrict__ h) {
@@ -221,7 +231,8 @@ combine_kernel(const T* __restrict__ u, const float* __restrict__ ysh, const T* 
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        t < Tn; t += warps) {
     // lane k < K holds row inv[t*K+k] and gate w[t*K+k]; shuffles hand them out
-    const int my_row = lane < K ? inv[t * K + lane] : 0;
+    // y rows: inv[t*K+k] (expert order) or t*K+k (token-slot order, inv NULL)
+    const int my_row = lane < K ? (inv ? inv[t * K + lane] : static_cast<int>(t * K + lane)) : 0;
     const float my_w = lane < K ? w[t * K + lane] : 0.0f;
     // the trip count is the same for every lane, so the shuffles stay converged
     for (int c0 = 0; c0 < d; c0 += 32 * V) {

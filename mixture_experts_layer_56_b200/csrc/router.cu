@@ -17,9 +17,10 @@ namespace moe {
 
 namespace {
 
-constexpr int kRouterWarps = 4;
+constexpr int kRouterWarps = 8;   // 4 token groups x 2 halves of d
+constexpr int kRouterThreads = kRouterWarps * 32;
 constexpr int kTokPerWarp = 8;
-constexpr int kTokPerCta = kRouterWarps * kTokPerWarp;  // 32
+constexpr int kTokPerCta = 4 * kTokPerWarp;  // 32
 
 // Eight consecutive elements of a row as fp32 (zero outside the matrix).
 template <typename TIn>
@@ -75,47 +76,53 @@ template <int EPT>
 constexpr int router_chunk() {
   return EPT <= 2 ? 128 : (EPT <= 4 ? 64 : 32);
 }
+constexpr int kPad = 4;  // floats of padding per staged row (bank spread)
 template <int EPT>
 constexpr int router_smem_bytes() {
-  return router_chunk<EPT>() * (kTokPerCta + EPT * 32) * 4;
+  return (kTokPerCta + EPT * 32) * (router_chunk<EPT>() + kPad) * 4;
 }
 
+// Two warps share each group of 8 tokens: warp w (< 4) sums the first half
+// of every d-chunk, warp w + 4 the second half; the two partial sums are
+// added once at the end (first half + second half), the same order for
+// every expert.
 template <typename TIn, int EPT, bool STATS>
-__global__ void __launch_bounds__(kRouterWarps * 32)
+__global__ void __launch_bounds__(kRouterThreads)
 router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
                    const float* __restrict__ bias, int64_t T, int d, int n, int K, int flags,
                    int32_t* __restrict__ idx, float* __restrict__ w, float* __restrict__ pstat) {
   constexpr int NP = EPT * 32;
   constexpr int KC = router_chunk<EPT>();
-  constexpr int NT = kRouterWarps * 32;      // threads
-  constexpr int UG = KC / 8 * kTokPerCta / NT;  // u items (8 columns each) per thread
-  constexpr int EG = KC / 8 * NP / NT;          // E items per thread
-  // one d-chunk of u (tokens) and E (experts), transposed to [j][row], fp32
+  constexpr int LD = KC + kPad;                  // staged row length (floats)
+  constexpr int NT = kRouterThreads;
+  constexpr int UI = KC / 8 * kTokPerCta;        // u items (8 columns each) per chunk
+  constexpr int EI = KC / 8 * NP;                // E items per chunk
+  constexpr int UG = (UI + NT - 1) / NT;         // items per thread
+  constexpr int EG = (EI + NT - 1) / NT;
+  // one d-chunk of u (tokens) and E (experts), row-major [row][j], fp32
   extern __shared__ __align__(16) float smem_f[];
-  float (*sU)[kTokPerCta] = reinterpret_cast<float (*)[kTokPerCta]>(smem_f);
-  float (*sE)[NP] = reinterpret_cast<float (*)[NP]>(smem_f + KC * kTokPerCta);
+  float* sU = smem_f;                  // [kTokPerCta][LD]
+  float* sE = smem_f + kTokPerCta * LD;  // [NP][LD]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  const int grp = warp & 3;        // token group of this warp
+  const int half = warp >> 2;      // which half of each chunk it sums
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTokPerCta;
 
-  // staging assignment: item i = tid + NT*k covers 8 columns of one row,
-  // row = i % rows, column group = i / rows.  Within a warp the group is
-  // fixed and the rows are consecutive, so the transposed stores hit 32
-  // distinct banks.
   Row8<TIn> pu[UG];
   Row8<TIn> pe[EG];
   auto prefetch = [&](int j0) {
 #pragma unroll
     for (int k = 0; k < UG; ++k) {
       const int i = tid + NT * k;
-      pu[k].load(u, t0 + i % kTokPerCta, T, d, j0 + (i / kTokPerCta) * 8);
+      if (UI % NT == 0 || i < UI) pu[k].load(u, t0 + i % kTokPerCta, T, d, j0 + (i / kTokPerCta) * 8);
     }
 #pragma unroll
     for (int k = 0; k < EG; ++k) {
       const int i = tid + NT * k;
-      pe[k].load(E, i % NP, n, d, j0 + (i / NP) * 8);
+      if (EI % NT == 0 || i < EI) pe[k].load(E, i % NP, n, d, j0 + (i / NP) * 8);
     }
   };
 
@@ -131,31 +138,69 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
 #pragma unroll
     for (int k = 0; k < UG; ++k) {
       const int i = tid + NT * k;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) sU[(i / kTokPerCta) * 8 + q][i % kTokPerCta] = pu[k].get(q);
+      if (UI % NT != 0 && i >= UI) continue;
+      float* dst = sU + (i % kTokPerCta) * LD + (i / kTokPerCta) * 8;
+      *reinterpret_cast<float4*>(dst) = make_float4(pu[k].get(0), pu[k].get(1), pu[k].get(2), pu[k].get(3));
+      *reinterpret_cast<float4*>(dst + 4) = make_float4(pu[k].get(4), pu[k].get(5), pu[k].get(6), pu[k].get(7));
     }
 #pragma unroll
     for (int k = 0; k < EG; ++k) {
       const int i = tid + NT * k;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) sE[(i / NP) * 8 + q][i % NP] = pe[k].get(q);
+      if (EI % NT != 0 && i >= EI) continue;
+      float* dst = sE + (i % NP) * LD + (i / NP) * 8;
+      *reinterpret_cast<float4*>(dst) = make_float4(pe[k].get(0), pe[k].get(1), pe[k].get(2), pe[k].get(3));
+      *reinterpret_cast<float4*>(dst + 4) = make_float4(pe[k].get(4), pe[k].get(5), pe[k].get(6), pe[k].get(7));
     }
     __syncthreads();
     if (j0 + KC < d) prefetch(j0 + KC);  // in flight during the FMAs below
-    const int jn = min(KC, d - j0);
-#pragma unroll 8
-    for (int j = 0; j < jn; ++j) {
-      float ev[EPT];
+    // columns past d were staged as zeros, so the products there are 0
+    const int jb = half * (KC / 2);
+    // shared-memory loads one step (4 columns) ahead of the FMAs that use them
+    float4 ev[2][EPT], uv[2][kTokPerWarp];
+    auto load_step = [&](int buf, int jj) {
 #pragma unroll
-      for (int q = 0; q < EPT; ++q) ev[q] = sE[j][lane + 32 * q];
-      const float4 ua = *reinterpret_cast<const float4*>(&sU[j][warp * kTokPerWarp]);
-      const float4 ub = *reinterpret_cast<const float4*>(&sU[j][warp * kTokPerWarp + 4]);
-      const float uv[kTokPerWarp] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+      for (int q = 0; q < EPT; ++q)
+        ev[buf][q] = *reinterpret_cast<const float4*>(sE + (lane + 32 * q) * LD + jb + jj);
 #pragma unroll
       for (int i = 0; i < kTokPerWarp; ++i)
+        uv[buf][i] = *reinterpret_cast<const float4*>(sU + (grp * kTokPerWarp + i) * LD + jb + jj);
+    };
+    load_step(0, 0);
 #pragma unroll
-        for (int q = 0; q < EPT; ++q) acc[i][q] = fmaf(uv[i], ev[q], acc[i][q]);
+    for (int jj = 0; jj < KC / 2; jj += 4) {
+      const int cur = (jj / 4) & 1;
+      if (jj + 4 < KC / 2) load_step(cur ^ 1, jj + 4);
+#pragma unroll
+      for (int i = 0; i < kTokPerWarp; ++i) {
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+          float a = acc[i][q];
+          a = fmaf(uv[cur][i].x, ev[cur][q].x, a);
+          a = fmaf(uv[cur][i].y, ev[cur][q].y, a);
+          a = fmaf(uv[cur][i].z, ev[cur][q].z, a);
+          a = fmaf(uv[cur][i].w, ev[cur][q].w, a);
+          acc[i][q] = a;
+        }
+      }
     }
+  }
+
+  // second-half partial sums -> first-half warps
+  __syncthreads();
+  float* red = smem_f;  // [4 warps][kTokPerWarp][EPT][32]
+  if (half == 1) {
+#pragma unroll
+    for (int i = 0; i < kTokPerWarp; ++i)
+#pragma unroll
+      for (int q = 0; q < EPT; ++q) red[((grp * kTokPerWarp + i) * EPT + q) * 32 + lane] = acc[i][q];
+  }
+  __syncthreads();
+  if (half == 0) {
+#pragma unroll
+    for (int i = 0; i < kTokPerWarp; ++i)
+#pragma unroll
+      for (int q = 0; q < EPT; ++q)
+        acc[i][q] += red[((grp * kTokPerWarp + i) * EPT + q) * 32 + lane];
   }
 
   float b[EPT];
@@ -170,10 +215,11 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
 #pragma unroll
   for (int q = 0; q < EPT; ++q) pst[q] = 0.0f;
 
+  // softmax and top-K: the first-half warps, one token at a time
 #pragma unroll
   for (int i = 0; i < kTokPerWarp; ++i) {
-    const int64_t t = t0 + warp * kTokPerWarp + i;
-    if (t >= T) break;  // warp-uniform
+    const int64_t t = t0 + grp * kTokPerWarp + i;
+    if (half != 0 || t >= T) break;  // warp-uniform
     // softmax logits (with the bias unless it only steers the selection)
     // and selection keys
     float lg[EPT], key[EPT];
@@ -240,13 +286,15 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
 
   if (STATS) {
     // per-CTA partial sums of the scores, reduced in a fixed order later
-    __shared__ float red[kRouterWarps][NP];
+    __shared__ float pred[4][NP];
+    if (half == 0) {
 #pragma unroll
-    for (int q = 0; q < EPT; ++q) red[warp][lane + 32 * q] = pst[q];
+      for (int q = 0; q < EPT; ++q) pred[grp][lane + 32 * q] = pst[q];
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < n; e += blockDim.x) {
       float a = 0.0f;
-      for (int ww = 0; ww < kRouterWarps; ++ww) a += red[ww][e];
+      for (int g = 0; g < 4; ++g) a += pred[g][e];
       pstat[static_cast<int64_t>(blockIdx.x) * n + e] = a;
     }
   }
@@ -257,7 +305,7 @@ int launch_router_t(const TIn* u, const TIn* E, const float* bias, int64_t T, in
                     int flags, int32_t* idx, float* w, float* pstat, cudaStream_t st) {
   const int ept = (n + 31) / 32;
   const unsigned grid = static_cast<unsigned>((T + kTokPerCta - 1) / kTokPerCta);
-  const dim3 block(kRouterWarps * 32);
+  const dim3 block(kRouterThreads);
 #define MOE_ROUTER_CASE(N)                                                                  \
   case N: {                                                                                 \
     auto kern = router_topk_kernel<TIn, N, STATS>;                                          \

@@ -39,10 +39,26 @@ def test_tiny_fp32_config_full():
     print(rep["near_ties"], rep["err_h"])
 
 
+GEMM_MODES = {"single_cta": L.MOE_FLAG_GEMM_SINGLE_CTA, "cta_pair": L.MOE_FLAG_GEMM_CTA_PAIR}
+
+
+@pytest.mark.parametrize("mode", sorted(GEMM_MODES))
 @pytest.mark.parametrize("wl", CASES, ids=[c.name for c in CASES])
-def test_bf16_cases_full(wl):
-    rep = P.full_parity(S.make_inputs(wl))
-    print(wl.name, {k: v for k, v in rep.items() if k != "gpu"})
+def test_bf16_cases_full(wl, mode):
+    rep = P.full_parity(S.make_inputs(wl), flags=GEMM_MODES[mode])
+    print(wl.name, mode, {k: v for k, v in rep.items() if k != "gpu"})
+
+
+@pytest.mark.parametrize("mode", sorted(GEMM_MODES))
+def test_gemm_tile_modes_agree(mode):
+    """Both tile shapes give results within the bf16 bar of each other and
+    the same routing (the routing does not depend on the GEMM)."""
+    wl = W("modes", T=900, d=256, n_routed=8, n_shared=1, inter=128, top_k=2)
+    x = S.make_inputs(wl)
+    a = P.gpu_stages(x, flags=GEMM_MODES[mode])
+    b = P.gpu_stages(x, flags=0)
+    assert np.array_equal(a["idx"], b["idx"])
+    P.assert_close(a["h"], b["h"], "h across tile modes")
 
 
 def test_every_expert_selected_sums_gates_to_one():
@@ -61,10 +77,11 @@ def test_empty_experts_from_skewed_bias():
     assert np.sum(rep["gpu"]["counts"] == 0) >= 8
 
 
-@pytest.mark.parametrize("T", [1, 2, 127, 128, 129])
-def test_token_counts_around_one_tile(T):
-    wl = W(f"t{T}", T=T, d=256, n_routed=16, n_shared=1, inter=128, top_k=4)
-    P.full_parity(S.make_inputs(wl))
+@pytest.mark.parametrize("mode", sorted(GEMM_MODES))
+@pytest.mark.parametrize("T", [1, 2, 127, 128, 129, 255, 256, 257])
+def test_token_counts_around_one_tile(T, mode):
+    wl = W(f"t{T}", T=T, d=256, n_routed=4, n_shared=1, inter=128, top_k=2)
+    P.full_parity(S.make_inputs(wl), flags=GEMM_MODES[mode])
 
 
 def test_duplicate_centroids_lower_index_wins():
