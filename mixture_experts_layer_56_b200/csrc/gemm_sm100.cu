@@ -81,6 +81,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+  // SwiGLU epilogues drain with 8 warps (two per TMEM lane quarter, one per
+  // half of the columns); plain ones with 4
+  constexpr int EPI_WARPS = EPI == kEpiSwiGLU ? 8 : 4;
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[2 * STAGES + 5];
@@ -115,7 +118,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 8);  // one arrive per epilogue warp
+      mbar_init(tempty_bar(a), EPI_WARPS);  // one arrive per epilogue warp
     }
     mbar_init(drain_bar, 1);
     abort_flag = 0;
@@ -247,7 +250,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 4 + EPI_WARPS) {
     // ------------------------------------------------------- epilogue -----
     const int q = warp & 3;          // TMEM lane quarter of this warp
     const int hcol = (warp - 4) >> 2;  // which half of the tile's columns it drains
@@ -273,7 +276,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
         const int64_t ld = ti.shared ? args.ld_s : args.ld_r;
         const int64_t col0 = static_cast<int64_t>(ti.n_blk) * (BN / 2);
 #pragma unroll 1
-        for (int c = hcol * (BN / 128); c < (hcol + 1) * (BN / 128); ++c) {
+        for (int c = hcol * (BN / 128); c < (hcol + 1) * (BN / 128); ++c) {  // 8 warps
           const int pair = c >> 1, half = c & 1;
           const int gcol = pair * 128 + half * 32;
           float gv[32], uv[32];
@@ -293,7 +296,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
         }
       } else {
 #pragma unroll 1
-        for (int c = hcol * (BN / 64); c < (hcol + 1) * (BN / 64); ++c) {
+        for (int c = 0; c < BN / 32; ++c) {  // 4 warps
           float x[32];
           tmem_ld32(taddr + c * 32, x);
           tmem_ld_wait();

@@ -31,14 +31,52 @@ constexpr int PBK = 64;
 constexpr int kPairThreads = 384;  // 4 role warps + 8 epilogue warps
 constexpr int kPairMaxGroups = 257;
 
-template <int BN> struct PairCfg;
-template <> struct PairCfg<256> { static constexpr int STAGES = 6; };
-template <> struct PairCfg<128> { static constexpr int STAGES = 8; };
-template <> struct PairCfg<64>  { static constexpr int STAGES = 9; };
+// Epilogue staging: every epilogue warp owns 32 rows x (128 + 16) bytes of
+// shared memory; rows are padded by 16 bytes so that 32 lanes writing one
+// row each hit distinct banks.
+constexpr int kStageRowBytes = 128;
+constexpr int kStagePitch = kStageRowBytes + 16;
+constexpr int kWarpStageBytes = 32 * kStagePitch;
 
-template <int BN>
+template <int EPI> constexpr int pair_epi_warps() { return EPI == kEpiSwiGLU ? 8 : 4; }
+
+// pipeline depth: as many 256-row k-block stages as fit beside the staging
+template <int BN, int EPI>
+constexpr int pair_stages() {
+  return (216 * 1024 - pair_epi_warps<EPI>() * kWarpStageBytes) /
+         (HBM_ROWS * PBK * 2 + (BN / 2) * PBK * 2);
+}
+
+template <int BN, int EPI>
 constexpr int pair_smem_bytes() {
-  return PairCfg<BN>::STAGES * (HBM_ROWS * PBK * 2 + (BN / 2) * PBK * 2) + 1024;
+  return pair_stages<BN, EPI>() * (HBM_ROWS * PBK * 2 + (BN / 2) * PBK * 2) +
+         pair_epi_warps<EPI>() * kWarpStageBytes + 1024;
+}
+
+// A warp's 32 rows of ROW_BYTES bytes each (lane r holds row r in `v`) go
+// to global memory through its shared staging area, as full row segments:
+// ROW_BYTES / 16 lanes write one row, so one store instruction covers
+// 512 / ROW_BYTES rows with whole 32-byte sectors.  `dst` is lane r's row
+// start (nullptr: row r is not written).
+template <int ROW_BYTES>
+__device__ __forceinline__ void warp_store_rows(uint8_t* stage, const uint4* v, uint8_t* dst,
+                                                int lane) {
+  constexpr int CH = ROW_BYTES / 16;  // 16-byte chunks per row
+  constexpr int RPI = 32 / CH;        // rows per store instruction
+#pragma unroll
+  for (int c = 0; c < CH; ++c)
+    *reinterpret_cast<uint4*>(stage + lane * kStagePitch + c * 16) = v[c];
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < CH; ++it) {
+    const int row = it * RPI + lane / CH;
+    const int c = lane % CH;
+    uint8_t* rdst = reinterpret_cast<uint8_t*>(
+        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), row));
+    const uint4 x = *reinterpret_cast<const uint4*>(stage + row * kStagePitch + c * 16);
+    if (rdst != nullptr) *reinterpret_cast<uint4*>(rdst + c * 16) = x;
+  }
+  __syncwarp();
 }
 
 struct PairTile {
@@ -68,12 +106,15 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                          const __grid_constant__ CUtensorMap tmA_s,
                          const __grid_constant__ CUtensorMap tmB_r,
                          const __grid_constant__ CUtensorMap tmB_s, const GroupedGemmArgs args) {
-  constexpr int STAGES = PairCfg<BN>::STAGES;
+  constexpr int STAGES = pair_stages<BN, EPI>();
   constexpr uint32_t A_BYTES = HBM_ROWS * PBK * 2;
   constexpr uint32_t B_BYTES = (BN / 2) * PBK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr uint32_t IDESC = idesc_bf16_f32(PBM, BN);
+  // SwiGLU epilogues drain with 8 warps (two per TMEM lane quarter, one per
+  // half of the columns); plain ones with 4
+  constexpr int EPI_WARPS = pair_epi_warps<EPI>();
   constexpr uint16_t kBoth = 0x3;
 
   extern __shared__ uint8_t smem_raw[];
@@ -113,7 +154,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);   // one multicast commit
-      mbar_init(tempty_bar(a), 16);  // 8 epilogue warps x 2 CTAs (leader's copy)
+      mbar_init(tempty_bar(a), 2 * EPI_WARPS);  // epilogue warps of both CTAs (leader's copy)
     }
     mbar_init(drain_bar, 1);
     abort_flag = 0;
@@ -237,7 +278,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 4 + EPI_WARPS) {
     // ------------------------------------------------------- epilogue -----
     const int q = warp & 3;          // TMEM lane quarter of this warp
     const int hcol = (warp - 4) >> 2;  // which half of the tile's columns it drains
@@ -262,46 +303,61 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                                : orow;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
+      uint8_t* stage = smem + STAGES * STAGE_BYTES + (warp - 4) * kWarpStageBytes;
       if (EPI == kEpiSwiGLU) {
+        // this warp's output columns: 64 (BN = 256) or 32 (BN = 128)
+        constexpr int OC = BN / 4;
         bf16* out = static_cast<bf16*>(ti.shared ? args.out_s : args.out_r);
         const int64_t ld = ti.shared ? args.ld_s : args.ld_r;
-        const int64_t col0 = static_cast<int64_t>(ti.n_blk) * (BN / 2);
-#pragma unroll 1
-        for (int c = hcol * (BN / 128); c < (hcol + 1) * (BN / 128); ++c) {
-          const int pair = c >> 1, half = c & 1;
-          const int gcol = pair * 128 + half * 32;
+        const int64_t col0 = static_cast<int64_t>(ti.n_blk) * (BN / 2) + hcol * OC;
+        uint4 packed[OC / 8];
+#pragma unroll
+        for (int h = 0; h < OC / 32; ++h) {
+          // packed blocks of 128 columns are [gate 64 | up 64]; this warp's
+          // gate columns start at 128*hcol (BN = 256) or 32*hcol (BN = 128)
+          const int gcol = (BN == 256 ? hcol * 128 : hcol * 32) + h * 32;
+          const int ucol = gcol + 64;
           float gv[32], uv[32];
           tmem_ld32(taddr + gcol, gv);
-          tmem_ld32(taddr + gcol + 64, uv);
+          tmem_ld32(taddr + ucol, uv);
           tmem_ld_wait();
-          if (live) {
-            bf16* dst = out + orow * ld + col0 + pair * 64 + half * 32;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              float o[8];
+          for (int v = 0; v < 4; ++v) {
+            float o[8];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) o[j] = silu_mul(gv[v * 8 + j], uv[v * 8 + j]);
-              Vec16<bf16>::store(dst + v * 8, o);
-            }
+            for (int j = 0; j < 8; ++j) o[j] = silu_mul(gv[v * 8 + j], uv[v * 8 + j]);
+            Vec16<bf16>::store(reinterpret_cast<bf16*>(&packed[h * 4 + v]), o);
           }
         }
+        uint8_t* dst = live ? reinterpret_cast<uint8_t*>(out + orow * ld + col0) : nullptr;
+        warp_store_rows<OC * 2>(stage, packed, dst, lane);
       } else {
 #pragma unroll 1
-        for (int c = hcol * (BN / 64); c < (hcol + 1) * (BN / 64); ++c) {
+        for (int c = 0; c < BN / 32; ++c) {
           float x[32];
           tmem_ld32(taddr + c * 32, x);
           tmem_ld_wait();
-          if (live) {
-            const int64_t col = static_cast<int64_t>(ti.n_blk) * BN + c * 32;
-            if (ti.shared) {
-              float* dst = static_cast<float*>(args.out_s) + orow * args.ld_s + col;
+          const int64_t col = static_cast<int64_t>(ti.n_blk) * BN + c * 32;
+          if (ti.shared) {
+            // fp32: 32 columns = 128 bytes per row
+            uint4 packed[8];
 #pragma unroll
-              for (int v = 0; v < 8; ++v) Vec16<float>::store(dst + v * 4, x + v * 4);
-            } else {
-              bf16* dst = static_cast<bf16*>(args.out_r) + prow * args.ld_r + col;
+            for (int v = 0; v < 8; ++v)
+              packed[v] = make_uint4(__float_as_uint(x[4 * v]), __float_as_uint(x[4 * v + 1]),
+                                     __float_as_uint(x[4 * v + 2]), __float_as_uint(x[4 * v + 3]));
+            uint8_t* dst = live ? reinterpret_cast<uint8_t*>(static_cast<float*>(args.out_s) +
+                                                             orow * args.ld_s + col)
+                                : nullptr;
+            warp_store_rows<128>(stage, packed, dst, lane);
+          } else {
+            // bf16: 32 columns = 64 bytes per row
+            uint4 packed[4];
 #pragma unroll
-              for (int v = 0; v < 4; ++v) Vec16<bf16>::store(dst + v * 8, x + v * 8);
-            }
+            for (int v = 0; v < 4; ++v) Vec16<bf16>::store(reinterpret_cast<bf16*>(&packed[v]), x + v * 8);
+            uint8_t* dst = live ? reinterpret_cast<uint8_t*>(static_cast<bf16*>(args.out_r) +
+                                                             prow * args.ld_r + col)
+                                : nullptr;
+            warp_store_rows<64>(stage, packed, dst, lane);
           }
         }
       }
@@ -326,14 +382,14 @@ int launch_pair_impl(const GemmMaps& m, const GroupedGemmArgs& args, int cluster
   auto kern = grouped_gemm_pair_kernel<BN, EPI>;
   if (!attr_done) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             pair_smem_bytes<BN>()) != cudaSuccess)
+                             pair_smem_bytes<BN, EPI>()) != cudaSuccess)
       return MOE_ERR_CUDA;
     attr_done = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(kPairThreads, 1, 1);
-  cfg.dynamicSmemBytes = pair_smem_bytes<BN>();
+  cfg.dynamicSmemBytes = pair_smem_bytes<BN, EPI>();
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

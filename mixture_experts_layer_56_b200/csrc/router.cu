@@ -21,6 +21,10 @@ constexpr int kRouterWarps = 8;   // 4 token groups x 2 halves of d
 constexpr int kRouterThreads = kRouterWarps * 32;
 constexpr int kTokPerWarp = 8;
 constexpr int kTokPerCta = 4 * kTokPerWarp;  // 32
+#ifndef MOE_ROUTER_LOOKAHEAD
+#define MOE_ROUTER_LOOKAHEAD 2
+#endif
+constexpr int kRouterLookahead = MOE_ROUTER_LOOKAHEAD;  // shared-load lookahead (d-steps)
 
 // Eight consecutive elements of a row as fp32 (zero outside the matrix).
 template <typename TIn>
@@ -70,138 +74,164 @@ struct Row8<float> {
   }
 };
 
-// d-chunk staged per step: as long as shared memory allows (the global loads
-// of the next chunk are in flight while the current one is multiplied).
+// d-chunk staged per step (the global loads of the next chunk are in flight
+// while the current one is multiplied).
 template <int EPT>
 constexpr int router_chunk() {
-  return EPT <= 2 ? 128 : (EPT <= 4 ? 64 : 32);
+  return EPT <= 4 ? 64 : 32;
 }
-constexpr int kPad = 4;  // floats of padding per staged row (bank spread)
 template <int EPT>
 constexpr int router_smem_bytes() {
-  return (kTokPerCta + EPT * 32) * (router_chunk<EPT>() + kPad) * 4;
+  return router_chunk<EPT>() * (kTokPerCta + EPT * 32) * 4;
 }
 
-// Two warps share each group of 8 tokens: warp w (< 4) sums the first half
-// of every d-chunk, warp w + 4 the second half; the two partial sums are
-// added once at the end (first half + second half), the same order for
-// every expert.
+// The logits of the CTA's 32 tokens x NP experts are an outer-product
+// register tile: thread h of a 128-thread half owns tokens 4*(h%8)..+3 and
+// experts XPT*(h/8)..+XPT-1 (XPT = 2*EPT), so one d-step costs it one
+// 16-byte load of token values, XPT/4 of expert values (each a single
+// shared-memory wavefront per warp) and 4*XPT FMAs.  The two halves of the
+// CTA sum the two halves of every d-chunk; their partial sums are added once
+// at the end (first half + second half), in the same order for every
+// expert, so equal centroids give equal logits.
 template <typename TIn, int EPT, bool STATS>
 __global__ void __launch_bounds__(kRouterThreads)
 router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
                    const float* __restrict__ bias, int64_t T, int d, int n, int K, int flags,
                    int32_t* __restrict__ idx, float* __restrict__ w, float* __restrict__ pstat) {
   constexpr int NP = EPT * 32;
+  constexpr int XPT = 2 * EPT;                   // experts per thread
   constexpr int KC = router_chunk<EPT>();
-  constexpr int LD = KC + kPad;                  // staged row length (floats)
   constexpr int NT = kRouterThreads;
   constexpr int UI = KC / 8 * kTokPerCta;        // u items (8 columns each) per chunk
   constexpr int EI = KC / 8 * NP;                // E items per chunk
   constexpr int UG = (UI + NT - 1) / NT;         // items per thread
   constexpr int EG = (EI + NT - 1) / NT;
-  // one d-chunk of u (tokens) and E (experts), row-major [row][j], fp32
+  constexpr int LDL = NP + 1;                    // logits row length (floats)
+  static_assert(KC * (kTokPerCta + NP) >= kTokPerCta * LDL, "logits fit the staging area");
+  // one d-chunk of u and E transposed to [j][row] (fp32); afterwards the
+  // [token][expert] logits
   extern __shared__ __align__(16) float smem_f[];
-  float* sU = smem_f;                  // [kTokPerCta][LD]
-  float* sE = smem_f + kTokPerCta * LD;  // [NP][LD]
+  float* sU = smem_f;                   // [KC][kTokPerCta]
+  float* sE = smem_f + KC * kTokPerCta;  // [KC][NP]
+  float* sL = smem_f;                   // [kTokPerCta][LDL]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int grp = warp & 3;        // token group of this warp
-  const int half = warp >> 2;      // which half of each chunk it sums
+  const int half = tid >> 7;            // which half of each chunk this thread sums
+  const int hh = tid & 127;
+  const int tg = hh & 7;                // tokens 4*tg .. 4*tg+3
+  const int eg = hh >> 3;               // experts XPT*eg .. XPT*eg+XPT-1
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTokPerCta;
 
-  Row8<TIn> pu[UG];
-  Row8<TIn> pe[EG];
-  auto prefetch = [&](int j0) {
+  // two register buffers of staged chunks: the global loads of chunk c+2
+  // are issued while chunk c is multiplied
+  struct Staged {
+    Row8<TIn> pu[UG];
+    Row8<TIn> pe[EG];
+  };
+  Staged bufA, bufB;
+  auto prefetch = [&](Staged& b, int j0) {
 #pragma unroll
     for (int k = 0; k < UG; ++k) {
       const int i = tid + NT * k;
-      if (UI % NT == 0 || i < UI) pu[k].load(u, t0 + i % kTokPerCta, T, d, j0 + (i / kTokPerCta) * 8);
+      if (UI % NT == 0 || i < UI) b.pu[k].load(u, t0 + i % kTokPerCta, T, d, j0 + (i / kTokPerCta) * 8);
     }
 #pragma unroll
     for (int k = 0; k < EG; ++k) {
       const int i = tid + NT * k;
-      if (EI % NT == 0 || i < EI) pe[k].load(E, i % NP, n, d, j0 + (i / NP) * 8);
+      if (EI % NT == 0 || i < EI) b.pe[k].load(E, i % NP, n, d, j0 + (i / NP) * 8);
     }
   };
 
-  float acc[kTokPerWarp][EPT];
+  float acc[4][XPT];
 #pragma unroll
-  for (int i = 0; i < kTokPerWarp; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int q = 0; q < EPT; ++q) acc[i][q] = 0.0f;
+    for (int m = 0; m < XPT; ++m) acc[i][m] = 0.0f;
 
-  prefetch(0);
-  for (int j0 = 0; j0 < d; j0 += KC) {
+  auto chunk = [&](Staged& b, int j0) {
     __syncthreads();  // the previous chunk's reads are done
+    // transposed stores: within a warp the 8-column group is fixed and the
+    // rows are consecutive, so each store hits 32 distinct banks
 #pragma unroll
     for (int k = 0; k < UG; ++k) {
       const int i = tid + NT * k;
       if (UI % NT != 0 && i >= UI) continue;
-      float* dst = sU + (i % kTokPerCta) * LD + (i / kTokPerCta) * 8;
-      *reinterpret_cast<float4*>(dst) = make_float4(pu[k].get(0), pu[k].get(1), pu[k].get(2), pu[k].get(3));
-      *reinterpret_cast<float4*>(dst + 4) = make_float4(pu[k].get(4), pu[k].get(5), pu[k].get(6), pu[k].get(7));
+#pragma unroll
+      for (int q = 0; q < 8; ++q) sU[((i / kTokPerCta) * 8 + q) * kTokPerCta + i % kTokPerCta] = b.pu[k].get(q);
     }
 #pragma unroll
     for (int k = 0; k < EG; ++k) {
       const int i = tid + NT * k;
       if (EI % NT != 0 && i >= EI) continue;
-      float* dst = sE + (i % NP) * LD + (i / NP) * 8;
-      *reinterpret_cast<float4*>(dst) = make_float4(pe[k].get(0), pe[k].get(1), pe[k].get(2), pe[k].get(3));
-      *reinterpret_cast<float4*>(dst + 4) = make_float4(pe[k].get(4), pe[k].get(5), pe[k].get(6), pe[k].get(7));
+#pragma unroll
+      for (int q = 0; q < 8; ++q) sE[((i / NP) * 8 + q) * NP + i % NP] = b.pe[k].get(q);
     }
     __syncthreads();
-    if (j0 + KC < d) prefetch(j0 + KC);  // in flight during the FMAs below
-    // columns past d were staged as zeros, so the products there are 0
+    if (j0 + 2 * KC < d) prefetch(b, j0 + 2 * KC);  // in flight during the next two chunks
+    // columns past d were staged as zeros, so their products are 0.  The
+    // shared-memory operands of step jj+1 are loaded before the FMAs of step
+    // jj, so their latency overlaps the arithmetic.
     const int jb = half * (KC / 2);
-    // shared-memory loads one step (4 columns) ahead of the FMAs that use them
-    float4 ev[2][EPT], uv[2][kTokPerWarp];
+    constexpr int LA = kRouterLookahead;  // d-steps of shared loads in flight
+    float ut[LA + 1][4], ev[LA + 1][XPT];
     auto load_step = [&](int buf, int jj) {
+      const float4 uv = *reinterpret_cast<const float4*>(sU + (jb + jj) * kTokPerCta + 4 * tg);
+      ut[buf][0] = uv.x; ut[buf][1] = uv.y; ut[buf][2] = uv.z; ut[buf][3] = uv.w;
+      if constexpr (XPT % 4 == 0) {
 #pragma unroll
-      for (int q = 0; q < EPT; ++q)
-        ev[buf][q] = *reinterpret_cast<const float4*>(sE + (lane + 32 * q) * LD + jb + jj);
+        for (int m = 0; m < XPT; m += 4) {
+          const float4 e4 = *reinterpret_cast<const float4*>(sE + (jb + jj) * NP + XPT * eg + m);
+          ev[buf][m] = e4.x; ev[buf][m + 1] = e4.y; ev[buf][m + 2] = e4.z; ev[buf][m + 3] = e4.w;
+        }
+      } else {
 #pragma unroll
-      for (int i = 0; i < kTokPerWarp; ++i)
-        uv[buf][i] = *reinterpret_cast<const float4*>(sU + (grp * kTokPerWarp + i) * LD + jb + jj);
-    };
-    load_step(0, 0);
-#pragma unroll
-    for (int jj = 0; jj < KC / 2; jj += 4) {
-      const int cur = (jj / 4) & 1;
-      if (jj + 4 < KC / 2) load_step(cur ^ 1, jj + 4);
-#pragma unroll
-      for (int i = 0; i < kTokPerWarp; ++i) {
-#pragma unroll
-        for (int q = 0; q < EPT; ++q) {
-          float a = acc[i][q];
-          a = fmaf(uv[cur][i].x, ev[cur][q].x, a);
-          a = fmaf(uv[cur][i].y, ev[cur][q].y, a);
-          a = fmaf(uv[cur][i].z, ev[cur][q].z, a);
-          a = fmaf(uv[cur][i].w, ev[cur][q].w, a);
-          acc[i][q] = a;
+        for (int m = 0; m < XPT; m += 2) {
+          const float2 e2 = *reinterpret_cast<const float2*>(sE + (jb + jj) * NP + XPT * eg + m);
+          ev[buf][m] = e2.x; ev[buf][m + 1] = e2.y;
         }
       }
+    };
+#pragma unroll
+    for (int l = 0; l < LA; ++l) load_step(l, l);
+#pragma unroll
+    for (int jj = 0; jj < KC / 2; ++jj) {
+      const int cur = jj % (LA + 1);
+      if (jj + LA < KC / 2) load_step((jj + LA) % (LA + 1), jj + LA);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int m = 0; m < XPT; ++m) acc[i][m] = fmaf(ut[cur][i], ev[cur][m], acc[i][m]);
     }
+  };
+
+  prefetch(bufA, 0);
+  if (KC < d) prefetch(bufB, KC);
+  for (int j0 = 0; j0 < d; j0 += 2 * KC) {
+    chunk(bufA, j0);
+    if (j0 + KC < d) chunk(bufB, j0 + KC);
   }
 
-  // second-half partial sums -> first-half warps
+  // logits = first-half sums + second-half sums, into [token][expert]
   __syncthreads();
-  float* red = smem_f;  // [4 warps][kTokPerWarp][EPT][32]
   if (half == 1) {
 #pragma unroll
-    for (int i = 0; i < kTokPerWarp; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int q = 0; q < EPT; ++q) red[((grp * kTokPerWarp + i) * EPT + q) * 32 + lane] = acc[i][q];
+      for (int m = 0; m < XPT; ++m) sL[(4 * tg + i) * LDL + XPT * eg + m] = acc[i][m];
   }
   __syncthreads();
   if (half == 0) {
 #pragma unroll
-    for (int i = 0; i < kTokPerWarp; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int q = 0; q < EPT; ++q)
-        acc[i][q] += red[((grp * kTokPerWarp + i) * EPT + q) * 32 + lane];
+      for (int m = 0; m < XPT; ++m) {
+        float* p = sL + (4 * tg + i) * LDL + XPT * eg + m;
+        *p = acc[i][m] + *p;
+      }
   }
+  __syncthreads();
 
   float b[EPT];
 #pragma unroll
@@ -215,19 +245,22 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
 #pragma unroll
   for (int q = 0; q < EPT; ++q) pst[q] = 0.0f;
 
-  // softmax and top-K: the first-half warps, one token at a time
-#pragma unroll
-  for (int i = 0; i < kTokPerWarp; ++i) {
-    const int64_t t = t0 + grp * kTokPerWarp + i;
-    if (half != 0 || t >= T) break;  // warp-uniform
+  // softmax and top-K: warp w takes tokens 4w..4w+3; lane L holds experts
+  // L, L+32, ...
+#pragma unroll 1
+  for (int i = 0; i < kTokPerCta / kRouterWarps; ++i) {
+    const int tl = warp * (kTokPerCta / kRouterWarps) + i;
+    const int64_t t = t0 + tl;
+    if (t >= T) break;  // warp-uniform
     // softmax logits (with the bias unless it only steers the selection)
     // and selection keys
     float lg[EPT], key[EPT];
 #pragma unroll
     for (int q = 0; q < EPT; ++q) {
       const int e = lane + 32 * q;
-      const float biased = acc[i][q] + b[q];
-      lg[q] = e < n ? (select_only ? acc[i][q] : biased) : -CUDART_INF_F;
+      const float l = sL[tl * LDL + e];
+      const float biased = l + b[q];
+      lg[q] = e < n ? (select_only ? l : biased) : -CUDART_INF_F;
       key[q] = e < n ? biased : -CUDART_INF_F;
     }
     float m = lg[0];
@@ -286,15 +319,14 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
 
   if (STATS) {
     // per-CTA partial sums of the scores, reduced in a fixed order later
-    __shared__ float pred[4][NP];
-    if (half == 0) {
+    __syncthreads();  // every warp is done reading the logits
+    float* pred = smem_f;  // [kRouterWarps][NP]
 #pragma unroll
-      for (int q = 0; q < EPT; ++q) pred[grp][lane + 32 * q] = pst[q];
-    }
+    for (int q = 0; q < EPT; ++q) pred[warp * NP + lane + 32 * q] = pst[q];
     __syncthreads();
     for (int e = threadIdx.x; e < n; e += blockDim.x) {
       float a = 0.0f;
-      for (int g = 0; g < 4; ++g) a += pred[g][e];
+      for (int ww = 0; ww < kRouterWarps; ++ww) a += pred[ww * NP + e];
       pstat[static_cast<int64_t>(blockIdx.x) * n + e] = a;
     }
   }
