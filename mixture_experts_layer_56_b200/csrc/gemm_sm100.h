@@ -39,6 +39,11 @@ bool make_map_bf16(CUtensorMap* map, int rank, const void* base, uint64_t inner,
                    uint64_t depth, uint64_t row_stride_bytes, uint64_t depth_stride_bytes,
                    uint32_t box_rows);
 
+// Rank-2 map with 128-byte swizzle: box {box_inner, box_rows}; the box's
+// inner extent must be 128 bytes.
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                 uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows);
+
 int launch_grouped_gemm(int BN, int epi, const GemmMaps& maps, const GroupedGemmArgs& args,
                         int grid, cudaStream_t stream);
 

@@ -2,147 +2,107 @@
 // l_{t,i} = sum_j u_{t,j} e_{i,j} (+ b_i) on CUDA cores, softmax over the
 // routed experts and top-K selection with warp shuffles.
 //
-// A CTA of 4 warps owns 32 tokens; a warp owns 8 tokens and lane L owns
-// experts L, L+32, ... (EPT = ceil(N_r / 32) of them).  d is walked in
-// 32-wide chunks staged in shared memory as fp32; every logit is one fp32
-// FMA chain in increasing j, so equal centroids give bitwise-equal logits.
-// The selection runs on logits (softmax is monotone), lower index first on
-// ties; gates are exp(l - max) / sum, not renormalised over the top K.
+// A CTA owns 32 tokens and all experts.  A producer warp streams 128-byte
+// column slices of u (32 rows) and E (NP rows) into a 4-stage shared-memory
+// ring with TMA (128-byte swizzle, rows past the matrix read as zeros), so
+// the loads of later slices are in flight while earlier ones are multiplied,
+// without costing registers.  The 256 compute threads form two halves; each
+// half sums one half of every slice, thread h owning the outer-product tile
+// tokens {h%8 + 8i} x experts {h/8 + 16m}, so a warp's shared loads are one
+// wavefront each.  Per logit every half is one fp32 FMA chain in increasing
+// j and the two halves are added once at the end, the same order for every
+// expert, so equal centroids give bitwise-equal logits.  The selection runs
+// on logits (softmax is monotone), lower index first on ties; gates are
+// exp(l - max) / sum, not renormalised over the top K.
+#include <cuda.h>
 #include <math_constants.h>
 
 #include "common.cuh"
+#include "gemm_sm100.h"
 #include "kernels.h"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kRouterWarps = 8;   // 4 token groups x 2 halves of d
-constexpr int kRouterThreads = kRouterWarps * 32;
-constexpr int kTokPerWarp = 8;
-constexpr int kTokPerCta = 4 * kTokPerWarp;  // 32
-#ifndef MOE_ROUTER_LOOKAHEAD
-#define MOE_ROUTER_LOOKAHEAD 2
-#endif
-constexpr int kRouterLookahead = MOE_ROUTER_LOOKAHEAD;  // shared-load lookahead (d-steps)
+using namespace sm100;
 
-// Eight consecutive elements of a row as fp32 (zero outside the matrix).
-template <typename TIn>
-struct Row8;
-template <>
-struct Row8<bf16> {
-  uint4 raw;
-  __device__ __forceinline__ void load(const bf16* __restrict__ src, int64_t row, int64_t nrows,
-                                       int d, int j) {
-    if (row < nrows && j + 8 <= d) {
-      raw = *reinterpret_cast<const uint4*>(src + row * d + j);
-    } else {
-      uint16_t h[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        h[q] = (row < nrows && j + q < d)
-                   ? reinterpret_cast<const uint16_t*>(src)[row * d + j + q] : uint16_t(0);
-      raw = make_uint4(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16),
-                       h[4] | (uint32_t(h[5]) << 16), h[6] | (uint32_t(h[7]) << 16));
-    }
-  }
-  __device__ __forceinline__ float get(int q) const {
-    const uint32_t w = q < 2 ? raw.x : q < 4 ? raw.y : q < 6 ? raw.z : raw.w;
-    return __uint_as_float((q & 1) ? (w & 0xffff0000u) : (w << 16));
-  }
-};
-template <>
-struct Row8<float> {
-  float4 lo, hi;
-  __device__ __forceinline__ void load(const float* __restrict__ src, int64_t row, int64_t nrows,
-                                       int d, int j) {
-    if (row < nrows && j + 8 <= d && (d & 3) == 0) {
-      lo = *reinterpret_cast<const float4*>(src + row * d + j);
-      hi = *reinterpret_cast<const float4*>(src + row * d + j + 4);
-    } else {
-      float v[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = (row < nrows && j + q < d) ? src[row * d + j + q] : 0.0f;
-      lo = make_float4(v[0], v[1], v[2], v[3]);
-      hi = make_float4(v[4], v[5], v[6], v[7]);
-    }
-  }
-  __device__ __forceinline__ float get(int q) const {
-    const float4& v = q < 4 ? lo : hi;
-    const int r = q & 3;
-    return r == 0 ? v.x : r == 1 ? v.y : r == 2 ? v.z : v.w;
-  }
-};
+constexpr int kRouterWarps = 8;                   // compute warps (two halves of 4)
+constexpr int kRouterThreads = kRouterWarps * 32 + 32;  // + one producer warp
+constexpr int kTokPerCta = 32;
+constexpr int kRouterStages = 4;
 
-// d-chunk staged per step (the global loads of the next chunk are in flight
-// while the current one is multiplied).
 template <int EPT>
-constexpr int router_chunk() {
-  return EPT <= 4 ? 64 : 32;
+constexpr int router_stage_bytes() {
+  return (kTokPerCta + EPT * 32) * 128;
 }
 template <int EPT>
 constexpr int router_smem_bytes() {
-  return router_chunk<EPT>() * (kTokPerCta + EPT * 32) * 4;
+  return kRouterStages * router_stage_bytes<EPT>() + 1024;
 }
 
-// The logits of the CTA's 32 tokens x NP experts are an outer-product
-// register tile: thread h of a 128-thread half owns tokens 4*(h%8)..+3 and
-// experts XPT*(h/8)..+XPT-1 (XPT = 2*EPT), so one d-step costs it one
-// 16-byte load of token values, XPT/4 of expert values (each a single
-// shared-memory wavefront per warp) and 4*XPT FMAs.  The two halves of the
-// CTA sum the two halves of every d-chunk; their partial sums are added once
-// at the end (first half + second half), in the same order for every
-// expert, so equal centroids give equal logits.
+// element v of a 16-byte chunk of 8 bf16 / 4 fp32 values, as fp32
+template <typename TIn>
+__device__ __forceinline__ float chunk_elem(const uint4& c, int v);
+template <>
+__device__ __forceinline__ float chunk_elem<bf16>(const uint4& c, int v) {
+  const uint32_t w = v < 2 ? c.x : v < 4 ? c.y : v < 6 ? c.z : c.w;
+  return __uint_as_float((v & 1) ? (w & 0xffff0000u) : (w << 16));
+}
+template <>
+__device__ __forceinline__ float chunk_elem<float>(const uint4& c, int v) {
+  return __uint_as_float(v == 0 ? c.x : v == 1 ? c.y : v == 2 ? c.z : c.w);
+}
+
+// 16-byte chunk ch of row `row` of a TMA tile with 128-byte rows and
+// 128-byte swizzle (tile base 1024-byte aligned)
+__device__ __forceinline__ uint4 lds_sw128(const uint8_t* tile, int row, int ch) {
+  return *reinterpret_cast<const uint4*>(tile + row * 128 + ((ch ^ (row & 7)) << 4));
+}
+
 template <typename TIn, int EPT, bool STATS>
 __global__ void __launch_bounds__(kRouterThreads)
-router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
+router_topk_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmE,
                    const float* __restrict__ bias, int64_t T, int d, int n, int K, int flags,
                    int32_t* __restrict__ idx, float* __restrict__ w, float* __restrict__ pstat) {
   constexpr int NP = EPT * 32;
-  constexpr int XPT = 2 * EPT;                   // experts per thread
-  constexpr int KC = router_chunk<EPT>();
-  constexpr int NT = kRouterThreads;
-  constexpr int UI = KC / 8 * kTokPerCta;        // u items (8 columns each) per chunk
-  constexpr int EI = KC / 8 * NP;                // E items per chunk
-  constexpr int UG = (UI + NT - 1) / NT;         // items per thread
-  constexpr int EG = (EI + NT - 1) / NT;
-  constexpr int LDL = NP + 1;                    // logits row length (floats)
-  static_assert(KC * (kTokPerCta + NP) >= kTokPerCta * LDL, "logits fit the staging area");
-  // one d-chunk of u and E transposed to [j][row] (fp32); afterwards the
-  // [token][expert] logits
-  extern __shared__ __align__(16) float smem_f[];
-  float* sU = smem_f;                   // [KC][kTokPerCta]
-  float* sE = smem_f + KC * kTokPerCta;  // [KC][NP]
-  float* sL = smem_f;                   // [kTokPerCta][LDL]
+  constexpr int XPT = 2 * EPT;                 // experts per thread
+  constexpr int VPC = 16 / sizeof(TIn);        // values per 16-byte chunk
+  constexpr int KC = 8 * VPC;                  // columns per stage (128-byte rows)
+  constexpr uint32_t U_BYTES = kTokPerCta * 128;
+  constexpr uint32_t ST_BYTES = router_stage_bytes<EPT>();
+  constexpr int LDL = NP + 1;                  // logits row length (floats)
+  static_assert(kRouterStages * ST_BYTES >= kTokPerCta * LDL * 4, "logits fit the ring");
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[2 * kRouterStages];
+  __shared__ int abort_flag;
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  float* sL = reinterpret_cast<float*>(ring);  // [kTokPerCta][LDL], after the d loop
+  const uint32_t ring_base = smem_addr(ring);
+  const uint32_t bar_base = smem_addr(bars);
+  auto full_bar = [&](int st) { return bar_base + 8u * st; };
+  auto empty_bar = [&](int st) { return bar_base + 8u * (kRouterStages + st); };
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int half = tid >> 7;            // which half of each chunk this thread sums
-  const int hh = tid & 127;
-  const int tg = hh & 7;                // tokens 4*tg .. 4*tg+3
-  const int eg = hh >> 3;               // experts XPT*eg .. XPT*eg+XPT-1
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTokPerCta;
+  const int nchunks = (d + KC - 1) / KC;
+  volatile int* abort_p = &abort_flag;
 
-  // two register buffers of staged chunks: the global loads of chunk c+2
-  // are issued while chunk c is multiplied
-  struct Staged {
-    Row8<TIn> pu[UG];
-    Row8<TIn> pe[EG];
-  };
-  Staged bufA, bufB;
-  auto prefetch = [&](Staged& b, int j0) {
-#pragma unroll
-    for (int k = 0; k < UG; ++k) {
-      const int i = tid + NT * k;
-      if (UI % NT == 0 || i < UI) b.pu[k].load(u, t0 + i % kTokPerCta, T, d, j0 + (i / kTokPerCta) * 8);
+  if (tid == 0) {
+    for (int st = 0; st < kRouterStages; ++st) {
+      mbar_init(full_bar(st), 1);
+      mbar_init(empty_bar(st), kRouterWarps);
     }
-#pragma unroll
-    for (int k = 0; k < EG; ++k) {
-      const int i = tid + NT * k;
-      if (EI % NT == 0 || i < EI) b.pe[k].load(E, i % NP, n, d, j0 + (i / NP) * 8);
-    }
-  };
+    abort_flag = 0;
+    fence_mbar_init();
+    fence_async_shared();
+  }
+  __syncthreads();
 
   float acc[4][XPT];
 #pragma unroll
@@ -150,84 +110,79 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
 #pragma unroll
     for (int m = 0; m < XPT; ++m) acc[i][m] = 0.0f;
 
-  auto chunk = [&](Staged& b, int j0) {
-    __syncthreads();  // the previous chunk's reads are done
-    // transposed stores: within a warp the 8-column group is fixed and the
-    // rows are consecutive, so each store hits 32 distinct banks
-#pragma unroll
-    for (int k = 0; k < UG; ++k) {
-      const int i = tid + NT * k;
-      if (UI % NT != 0 && i >= UI) continue;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) sU[((i / kTokPerCta) * 8 + q) * kTokPerCta + i % kTokPerCta] = b.pu[k].get(q);
+  if (warp == kRouterWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmU);
+      tma_prefetch_desc(&tmE);
+      for (int c = 0; c < nchunks; ++c) {
+        const int st = c % kRouterStages;
+        const uint32_t ph = (c / kRouterStages) & 1;
+        if (!wait_bounded(empty_bar(st), ph ^ 1u, abort_p, nullptr)) break;
+        const uint32_t sb = ring_base + st * ST_BYTES;
+        mbar_arrive_expect_tx(full_bar(st), ST_BYTES);
+        tma_load_2d(sb, &tmU, full_bar(st), c * KC, static_cast<int32_t>(t0));
+        tma_load_2d(sb + U_BYTES, &tmE, full_bar(st), c * KC, 0);
+      }
     }
+    __syncwarp();
+  } else {
+    // --------------------------------------------------------------- FMAs
+    const int half = tid >> 7;  // which 4 of the 8 chunks of every slice
+    const int hh = tid & 127;
+    const int tg = hh & 7;      // tokens tg + 8i
+    const int eg = hh >> 3;     // experts eg + 16m
+    for (int c = 0; c < nchunks; ++c) {
+      const int st = c % kRouterStages;
+      const uint32_t ph = (c / kRouterStages) & 1;
+      if (!wait_bounded(full_bar(st), ph, abort_p, nullptr)) break;
+      const uint8_t* uT = ring + st * ST_BYTES;
+      const uint8_t* eT = uT + U_BYTES;
 #pragma unroll
-    for (int k = 0; k < EG; ++k) {
-      const int i = tid + NT * k;
-      if (EI % NT != 0 && i >= EI) continue;
+      for (int q = 0; q < 4; ++q) {
+        const int ch = half * 4 + q;
+        uint4 ur[4], er[XPT];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) sE[((i / NP) * 8 + q) * NP + i % NP] = b.pe[k].get(q);
-    }
-    __syncthreads();
-    if (j0 + 2 * KC < d) prefetch(b, j0 + 2 * KC);  // in flight during the next two chunks
-    // columns past d were staged as zeros, so their products are 0.  The
-    // shared-memory operands of step jj+1 are loaded before the FMAs of step
-    // jj, so their latency overlaps the arithmetic.
-    const int jb = half * (KC / 2);
-    constexpr int LA = kRouterLookahead;  // d-steps of shared loads in flight
-    float ut[LA + 1][4], ev[LA + 1][XPT];
-    auto load_step = [&](int buf, int jj) {
-      const float4 uv = *reinterpret_cast<const float4*>(sU + (jb + jj) * kTokPerCta + 4 * tg);
-      ut[buf][0] = uv.x; ut[buf][1] = uv.y; ut[buf][2] = uv.z; ut[buf][3] = uv.w;
-      if constexpr (XPT % 4 == 0) {
+        for (int i = 0; i < 4; ++i) ur[i] = lds_sw128(uT, tg + 8 * i, ch);
 #pragma unroll
-        for (int m = 0; m < XPT; m += 4) {
-          const float4 e4 = *reinterpret_cast<const float4*>(sE + (jb + jj) * NP + XPT * eg + m);
-          ev[buf][m] = e4.x; ev[buf][m + 1] = e4.y; ev[buf][m + 2] = e4.z; ev[buf][m + 3] = e4.w;
-        }
-      } else {
+        for (int m = 0; m < XPT; ++m) er[m] = lds_sw128(eT, eg + 16 * m, ch);
 #pragma unroll
-        for (int m = 0; m < XPT; m += 2) {
-          const float2 e2 = *reinterpret_cast<const float2*>(sE + (jb + jj) * NP + XPT * eg + m);
-          ev[buf][m] = e2.x; ev[buf][m + 1] = e2.y;
+        for (int v = 0; v < VPC; ++v) {
+          float uf[4], ef[XPT];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) uf[i] = chunk_elem<TIn>(ur[i], v);
+#pragma unroll
+          for (int m = 0; m < XPT; ++m) ef[m] = chunk_elem<TIn>(er[m], v);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int m = 0; m < XPT; ++m) acc[i][m] = fmaf(uf[i], ef[m], acc[i][m]);
         }
       }
-    };
-#pragma unroll
-    for (int l = 0; l < LA; ++l) load_step(l, l);
-#pragma unroll
-    for (int jj = 0; jj < KC / 2; ++jj) {
-      const int cur = jj % (LA + 1);
-      if (jj + LA < KC / 2) load_step((jj + LA) % (LA + 1), jj + LA);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int m = 0; m < XPT; ++m) acc[i][m] = fmaf(ut[cur][i], ev[cur][m], acc[i][m]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(st));
     }
-  };
-
-  prefetch(bufA, 0);
-  if (KC < d) prefetch(bufB, KC);
-  for (int j0 = 0; j0 < d; j0 += 2 * KC) {
-    chunk(bufA, j0);
-    if (j0 + KC < d) chunk(bufB, j0 + KC);
   }
 
   // logits = first-half sums + second-half sums, into [token][expert]
-  __syncthreads();
-  if (half == 1) {
+  __syncthreads();  // every stage consumed; the ring is free
+  const int half = tid >> 7;
+  const int hh = tid & 127;
+  const int tg = hh & 7;
+  const int eg = hh >> 3;
+  if (warp < kRouterWarps && half == 1) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int m = 0; m < XPT; ++m) sL[(4 * tg + i) * LDL + XPT * eg + m] = acc[i][m];
+      for (int m = 0; m < XPT; ++m) sL[(tg + 8 * i) * LDL + eg + 16 * m] = acc[i][m];
   }
   __syncthreads();
-  if (half == 0) {
+  if (warp < kRouterWarps && half == 0) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int m = 0; m < XPT; ++m) {
-        float* p = sL + (4 * tg + i) * LDL + XPT * eg + m;
+        float* p = sL + (tg + 8 * i) * LDL + eg + 16 * m;
         *p = acc[i][m] + *p;
       }
   }
@@ -251,7 +206,7 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
   for (int i = 0; i < kTokPerCta / kRouterWarps; ++i) {
     const int tl = warp * (kTokPerCta / kRouterWarps) + i;
     const int64_t t = t0 + tl;
-    if (t >= T) break;  // warp-uniform
+    if (warp >= kRouterWarps || t >= T) break;  // warp-uniform; the producer has no tokens
     // softmax logits (with the bias unless it only steers the selection)
     // and selection keys
     float lg[EPT], key[EPT];
@@ -320,9 +275,11 @@ router_topk_kernel(const TIn* __restrict__ u, const TIn* __restrict__ E,
   if (STATS) {
     // per-CTA partial sums of the scores, reduced in a fixed order later
     __syncthreads();  // every warp is done reading the logits
-    float* pred = smem_f;  // [kRouterWarps][NP]
+    float* pred = sL;  // [kRouterWarps][NP]
+    if (warp < kRouterWarps) {
 #pragma unroll
-    for (int q = 0; q < EPT; ++q) pred[warp * NP + lane + 32 * q] = pst[q];
+      for (int q = 0; q < EPT; ++q) pred[warp * NP + lane + 32 * q] = pst[q];
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < n; e += blockDim.x) {
       float a = 0.0f;
@@ -338,13 +295,22 @@ int launch_router_t(const TIn* u, const TIn* E, const float* bias, int64_t T, in
   const int ept = (n + 31) / 32;
   const unsigned grid = static_cast<unsigned>((T + kTokPerCta - 1) / kTokPerCta);
   const dim3 block(kRouterThreads);
+  constexpr int VPC = 16 / sizeof(TIn);
+  const CUtensorMapDataType dt =
+      sizeof(TIn) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUtensorMap mu, me;
+  if (!make_map_2d(&mu, dt, u, static_cast<uint64_t>(d), static_cast<uint64_t>(T),
+                   static_cast<uint64_t>(d) * sizeof(TIn), 8 * VPC, kTokPerCta) ||
+      !make_map_2d(&me, dt, E, static_cast<uint64_t>(d), static_cast<uint64_t>(n),
+                   static_cast<uint64_t>(d) * sizeof(TIn), 8 * VPC, 32 * ept))
+    return MOE_ERR_CUDA;
 #define MOE_ROUTER_CASE(N)                                                                  \
   case N: {                                                                                 \
     auto kern = router_topk_kernel<TIn, N, STATS>;                                          \
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,             \
                              router_smem_bytes<N>()) != cudaSuccess)                        \
       return MOE_ERR_CUDA;                                                                  \
-    kern<<<grid, block, router_smem_bytes<N>(), st>>>(u, E, bias, T, d, n, K, flags, idx, w, \
+    kern<<<grid, block, router_smem_bytes<N>(), st>>>(mu, me, bias, T, d, n, K, flags, idx, w, \
                                                      pstat);                                \
     break;                                                                                  \
   }
