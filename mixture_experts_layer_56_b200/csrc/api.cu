@@ -111,7 +111,9 @@ Layout layout_of(const moe_shape_t& s) {
   L.chunk_counts = take(nch * n * 4);
   L.chunk_base = take(nch * n * 4);
   L.pstat = take(nrc * n * 4);
-  L.xperm = take(T * K * d * el);
+  // gathered rows are not materialised when the GEMM gathers them itself
+  const bool tma_gather = s.dtype == MOE_DTYPE_BF16 && (s.flags & MOE_FLAG_GEMM_TMA_GATHER);
+  L.xperm = take(tma_gather ? 0 : T * K * d * el);
   L.act = take(T * K * I * el);
   L.act_s = take(T * ns * I * el);
   L.y = take(T * K * d * el);
@@ -130,7 +132,8 @@ int validate(const moe_shape_t* s) {
       s->top_k > s->n_routed || s->top_k > 32 || s->n_shared < 0 || s->n_shared > 64 ||
       s->inter < 1)
     return MOE_ERR_SHAPE;
-  const int32_t known = MOE_FLAG_BIAS_SELECT_ONLY | MOE_FLAG_GEMM_SINGLE_CTA | MOE_FLAG_GEMM_CTA_PAIR;
+  const int32_t known = MOE_FLAG_BIAS_SELECT_ONLY | MOE_FLAG_GEMM_SINGLE_CTA |
+                        MOE_FLAG_GEMM_CTA_PAIR | MOE_FLAG_GEMM_TMA_GATHER;
   if ((s->flags & ~known) != 0) return MOE_ERR_SHAPE;
   if ((s->flags & MOE_FLAG_GEMM_SINGLE_CTA) && (s->flags & MOE_FLAG_GEMM_CTA_PAIR))
     return MOE_ERR_SHAPE;
@@ -190,7 +193,9 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
   void* xperm = at<void>(ws, L.xperm);
   void* act = at<void>(ws, L.act);
   void* act_s = at<void>(ws, L.act_s);
-  {
+  const bool tma_gather = s.dtype == MOE_DTYPE_BF16 && (s.flags & MOE_FLAG_GEMM_TMA_GATHER);
+  if (!tma_gather) {
+    // expert-sorted copies of the routed token rows
     Stage sg(MOE_KERNEL_GATHER, st);
     if (int rc = launch_gather(s.dtype, u, perm, rows, d, static_cast<int>(K), xperm, st))
       return rc;
@@ -237,7 +242,11 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     const int BN = (2 * I) % 256 == 0 ? 256 : 128;
     const uint32_t bbox = pair ? BN / 2 : BN;
     GemmMaps m;
-    bool ok = make_map_bf16(&m.a_r, 2, xperm, d64, rows, 1, d64 * 2, 0, 128) &&
+    // routed A rows: the expert-sorted copies, or token rows of u gathered
+    // through one-row boxes
+    bool ok = make_map_bf16(&m.a_g, 2, u, d64, T, 1, d64 * 2, 0, 1) &&
+              make_map_bf16(&m.a_r, 2, tma_gather ? u : xperm, d64, tma_gather ? T : rows, 1,
+                            d64 * 2, 0, 128) &&
               make_map_bf16(&m.b_r, 3, W13, d64, 2 * I64, n, d64 * 2, 2 * I64 * d64 * 2, bbox);
     if (ns > 0) {
       ok = ok && make_map_bf16(&m.a_s, 2, u, d64, T, 1, d64 * 2, 0, 128) &&
@@ -262,6 +271,8 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     a.out_s = act_s;
     a.ld_s = static_cast<int64_t>(I) * ns;
     a.status = status;
+    a.gather_perm = tma_gather ? perm : nullptr;
+    a.gather_k = static_cast<int32_t>(K);
     Stage sg(MOE_KERNEL_GEMM_GATE_UP, st);
     if (int rc = launch(BN, kEpiSwiGLU, m, a)) return rc;
   }
@@ -271,6 +282,7 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     const uint32_t bbox = pair ? BN / 2 : BN;
     GemmMaps m;
     bool ok = make_map_bf16(&m.a_r, 2, act, I64, rows, 1, I64 * 2, 0, 128) &&
+              make_map_bf16(&m.a_g, 2, act, I64, rows, 1, I64 * 2, 0, 1) &&
               make_map_bf16(&m.b_r, 3, W2, I64, d64, n, I64 * 2, d64 * I64 * 2, bbox);
     if (ns > 0) {
       ok = ok && make_map_bf16(&m.a_s, 2, act_s, I64 * ns, T, 1, I64 * ns * 2, 0, 128) &&
