@@ -259,9 +259,28 @@ def run_ours(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def forward():
+        # the stream current at call time (a graph capture switches it)
         L.moe_layer_forward(layer.shape, u, layer.E, layer.bias, layer.W13, layer.W2,
-                            layer.W13_s, layer.W2_s, h, layer.ws, stream=stream)
+                            layer.W13_s, layer.W2_s, h, layer.ws,
+                            stream=torch.cuda.current_stream(dev))
+
+    graph = None
+    if args.graph:
+        # one forward captured once and replayed per step: the C ABI only
+        # enqueues work on the caller's stream, so it captures as is
+        forward()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            forward()
+        torch.cuda.synchronize(dev)
+
+    def step():
+        if graph is not None:
+            graph.replay()
+        else:
+            forward()
 
     def barrier():
         if world > 1:
@@ -284,6 +303,12 @@ def run_ours(args):
             ends[i].record(stream)
         barrier()
     launches = L.moe_launch_count() - launches0
+    if graph is not None:
+        # replays bypass the library's launch counter: count one eager step
+        c0 = L.moe_launch_count()
+        forward()
+        torch.cuda.synchronize(dev)
+        launches = (L.moe_launch_count() - c0) * args.steps
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), dev)
     assert layer.status() == 0
@@ -297,7 +322,7 @@ def run_ours(args):
     prof_steps = 5
     for _ in range(prof_steps):
         flush.zero_()
-        step()
+        forward()
     torch.cuda.synchronize(dev)
     recs = L.moe_profile_read()
     L.moe_profile_enable(False)
@@ -364,7 +389,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic",
             "config": {"workload": workload_desc(wl), "tokens_per_gpu_step": wl.T,
-                       "gemm_tiles": args.gemm,
+                       "gemm_tiles": args.gemm, "cuda_graph": bool(args.graph),
                        "parallelism": f"replicas x{world} (token batches, no collective)",
                        "l2": "flushed between steps (256 MB memset outside the step events)",
                        "init": "seeded splitmix64/Box-Muller normals, bf16"},
@@ -410,6 +435,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step from a captured CUDA graph")
     ap.add_argument("--gemm", default="auto", choices=["auto", "single", "pair"],
                     help="tile shape of the expert GEMMs (default: chosen by the library)")
     args = ap.parse_args()

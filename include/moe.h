@@ -79,13 +79,6 @@ enum {
      same up to fp32 summation order inside the tensor cores. */
   MOE_FLAG_GEMM_SINGLE_CTA = 2,
   MOE_FLAG_GEMM_CTA_PAIR = 4,
-  /* bf16 gate/up GEMM: read the routed token rows straight from u with TMA
-     four-row gathers (tile::gather4) instead of first copying them into an
-     expert-sorted buffer.  Same results; it saves the copy and its
-     workspace, but 32 small gathers per 64-column k-block run the TMA unit
-     slower than the copy costs on B200 at the shapes measured here, so it is
-     off by default. */
-  MOE_FLAG_GEMM_TMA_GATHER = 8,
 };
 
 /* Layer shape.  Limits: 1 <= n_routed <= 256, 1 <= top_k <= min(n_routed, 32),

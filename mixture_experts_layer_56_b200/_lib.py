@@ -19,7 +19,6 @@ MOE_DTYPE_BF16 = 1
 MOE_FLAG_BIAS_SELECT_ONLY = 1
 MOE_FLAG_GEMM_SINGLE_CTA = 2
 MOE_FLAG_GEMM_CTA_PAIR = 4
-MOE_FLAG_GEMM_TMA_GATHER = 8
 
 MOE_OK = 0
 MOE_ERR_NULLPTR = -1

@@ -111,9 +111,7 @@ Layout layout_of(const moe_shape_t& s) {
   L.chunk_counts = take(nch * n * 4);
   L.chunk_base = take(nch * n * 4);
   L.pstat = take(nrc * n * 4);
-  // gathered rows are not materialised when the GEMM gathers them itself
-  const bool tma_gather = s.dtype == MOE_DTYPE_BF16 && (s.flags & MOE_FLAG_GEMM_TMA_GATHER);
-  L.xperm = take(tma_gather ? 0 : T * K * d * el);
+  L.xperm = take(T * K * d * el);
   L.act = take(T * K * I * el);
   L.act_s = take(T * ns * I * el);
   L.y = take(T * K * d * el);
@@ -133,7 +131,7 @@ int validate(const moe_shape_t* s) {
       s->inter < 1)
     return MOE_ERR_SHAPE;
   const int32_t known = MOE_FLAG_BIAS_SELECT_ONLY | MOE_FLAG_GEMM_SINGLE_CTA |
-                        MOE_FLAG_GEMM_CTA_PAIR | MOE_FLAG_GEMM_TMA_GATHER;
+                        MOE_FLAG_GEMM_CTA_PAIR;
   if ((s->flags & ~known) != 0) return MOE_ERR_SHAPE;
   if ((s->flags & MOE_FLAG_GEMM_SINGLE_CTA) && (s->flags & MOE_FLAG_GEMM_CTA_PAIR))
     return MOE_ERR_SHAPE;
@@ -193,8 +191,7 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
   void* xperm = at<void>(ws, L.xperm);
   void* act = at<void>(ws, L.act);
   void* act_s = at<void>(ws, L.act_s);
-  const bool tma_gather = s.dtype == MOE_DTYPE_BF16 && (s.flags & MOE_FLAG_GEMM_TMA_GATHER);
-  if (!tma_gather) {
+  {
     // expert-sorted copies of the routed token rows
     Stage sg(MOE_KERNEL_GATHER, st);
     if (int rc = launch_gather(s.dtype, u, perm, rows, d, static_cast<int>(K), xperm, st))
@@ -237,16 +234,22 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     return launch_grouped_gemm(BN, epi, m, a, static_cast<int>(grid), st);
   };
 
+  // the widest tile whose tile count still covers every SM (single-CTA
+  // tiles only: decode-sized batches need the extra parallelism)
+  auto pick_bn = [&](int n_cols_r, int n_cols_s, int widest, int narrowest) {
+    int bn = widest;
+    while (!pair && bn > narrowest && (n_cols_r % bn == 0) &&
+           routed_mt_ub * (n_cols_r / bn) + shared_mt * (n_cols_s / bn) < sms)
+      bn /= 2;
+    return bn;
+  };
+
   // ---- gate/up + SwiGLU ---------------------------------------------------
   {
-    const int BN = (2 * I) % 256 == 0 ? 256 : 128;
+    const int BN = pick_bn(2 * I, 2 * I * ns, (2 * I) % 256 == 0 ? 256 : 128, 128);
     const uint32_t bbox = pair ? BN / 2 : BN;
     GemmMaps m;
-    // routed A rows: the expert-sorted copies, or token rows of u gathered
-    // through one-row boxes
-    bool ok = make_map_bf16(&m.a_g, 2, u, d64, T, 1, d64 * 2, 0, 1) &&
-              make_map_bf16(&m.a_r, 2, tma_gather ? u : xperm, d64, tma_gather ? T : rows, 1,
-                            d64 * 2, 0, 128) &&
+    bool ok = make_map_bf16(&m.a_r, 2, xperm, d64, rows, 1, d64 * 2, 0, 128) &&
               make_map_bf16(&m.b_r, 3, W13, d64, 2 * I64, n, d64 * 2, 2 * I64 * d64 * 2, bbox);
     if (ns > 0) {
       ok = ok && make_map_bf16(&m.a_s, 2, u, d64, T, 1, d64 * 2, 0, 128) &&
@@ -271,18 +274,15 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     a.out_s = act_s;
     a.ld_s = static_cast<int64_t>(I) * ns;
     a.status = status;
-    a.gather_perm = tma_gather ? perm : nullptr;
-    a.gather_k = static_cast<int32_t>(K);
     Stage sg(MOE_KERNEL_GEMM_GATE_UP, st);
     if (int rc = launch(BN, kEpiSwiGLU, m, a)) return rc;
   }
   // ---- down projection ----------------------------------------------------
   {
-    const int BN = d % 256 == 0 ? 256 : (d % 128 == 0 ? 128 : 64);
+    const int BN = pick_bn(d, d, d % 256 == 0 ? 256 : (d % 128 == 0 ? 128 : 64), 64);
     const uint32_t bbox = pair ? BN / 2 : BN;
     GemmMaps m;
     bool ok = make_map_bf16(&m.a_r, 2, act, I64, rows, 1, I64 * 2, 0, 128) &&
-              make_map_bf16(&m.a_g, 2, act, I64, rows, 1, I64 * 2, 0, 1) &&
               make_map_bf16(&m.b_r, 3, W2, I64, d64, n, I64 * 2, d64 * I64 * 2, bbox);
     if (ns > 0) {
       ok = ok && make_map_bf16(&m.a_s, 2, act_s, I64 * ns, T, 1, I64 * ns * 2, 0, 128) &&

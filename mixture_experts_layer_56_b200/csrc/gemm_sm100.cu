@@ -74,7 +74,7 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
                     const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
-                    const __grid_constant__ CUtensorMap tmA_g, const GroupedGemmArgs args) {
+                    const GroupedGemmArgs args) {
   constexpr int STAGES = Cfg<BN>::STAGES;
   constexpr uint32_t A_BYTES = BM * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
@@ -171,8 +171,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
 
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer ----
-    // lane 0 owns the barriers and the tile loads; when routed A rows are
-    // gathered, every lane also issues one 4-row gather per k-block
     if (lane == 0) {
       tma_prefetch_desc(&tmA_r);
       tma_prefetch_desc(&tmB_r);
@@ -180,57 +178,38 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
         tma_prefetch_desc(&tmA_s);
         tma_prefetch_desc(&tmB_s);
       }
-      if (args.gather_perm) tma_prefetch_desc(&tmA_g);
-    }
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t issued = 0, issued_parity = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-      const TileInfo ti = decode_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
-      const CUtensorMap* ma = ti.shared ? &tmA_s : &tmA_r;
-      const CUtensorMap* mb = ti.shared ? &tmB_s : &tmB_r;
-      const int row = grp_row0[ti.g] + ti.m_blk * BM;
-      const int nrow = ti.n_blk * BN;
-      const int nkb = ti.shared ? args.kb_shared : args.kb_routed;
-      const int zbase = ti.shared ? 0 : ti.g - hs;
-      const bool gath = !ti.shared && args.gather_perm != nullptr;
-      int tok[4] = {0, 0, 0, 0};
-      if (gath) {
-        const int valid = grp_rows[ti.g] - ti.m_blk * BM;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int rr = 4 * lane + j;
-          tok[j] = rr < valid ? args.gather_perm[row + rr] / args.gather_k : 0;
-        }
-      }
-      for (int kb = 0; kb < nkb; ++kb) {
-        int got = 1;
-        if (lane == 0) got = wait_bounded(empty_bar(stage), phase ^ 1u, abort_p, args.status) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
-        const uint32_t sa = smem_base + stage * STAGE_BYTES;
-        if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        const TileInfo ti = decode_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+        const CUtensorMap* ma = ti.shared ? &tmA_s : &tmA_r;
+        const CUtensorMap* mb = ti.shared ? &tmB_s : &tmB_r;
+        const int row = grp_row0[ti.g] + ti.m_blk * BM;
+        const int nrow = ti.n_blk * BN;
+        const int nkb = ti.shared ? args.kb_shared : args.kb_routed;
+        const int zbase = ti.shared ? 0 : ti.g - hs;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_p, args.status)) { ok = false; break; }
+          const uint32_t sa = smem_base + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
-          if (!gath) tma_load_2d(sa, ma, full_bar(stage), kb * BK, row);
+          tma_load_2d(sa, ma, full_bar(stage), kb * BK, row);
           tma_load_3d(sa + A_BYTES, mb, full_bar(stage), (kb % args.kb_per_expert) * BK, nrow,
                       zbase + kb / args.kb_per_expert);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        __syncwarp();
-        if (gath)
-          tma_gather4(sa + lane * 512, &tmA_g, full_bar(stage), kb * BK, tok[0], tok[1], tok[2],
-                      tok[3]);
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-    }
-    if (!ok && lane == 0) {
-      // let every load already in flight land before the CTA exits
-      for (int s = 0; s < STAGES; ++s)
-        if (issued & (1u << s)) {
-          int dummy = 0;
-          wait_bounded(full_bar(s), (issued_parity >> s) & 1u, &dummy, nullptr);
-        }
+      if (!ok) {
+        // let every load already in flight land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) {
+            int dummy = 0;
+            wait_bounded(full_bar(s), (issued_parity >> s) & 1u, &dummy, nullptr);
+          }
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -408,7 +387,7 @@ static int launch_impl(const GemmMaps& m, const GroupedGemmArgs& args, int grid,
       return MOE_ERR_CUDA;
     attr_done = true;
   }
-  kern<<<grid, kThreads, smem_bytes<BN>(), stream>>>(m.a_r, m.a_s, m.b_r, m.b_s, m.a_g, args);
+  kern<<<grid, kThreads, smem_bytes<BN>(), stream>>>(m.a_r, m.a_s, m.b_r, m.b_s, args);
   count_launch();
   return check_launch();
 }

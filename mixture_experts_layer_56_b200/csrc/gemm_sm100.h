@@ -27,17 +27,12 @@ struct GroupedGemmArgs {
   void* out_s;             // shared output: bf16 (SwiGLU) or fp32 (plain)
   int64_t ld_s;
   int32_t* status;         // workspace status word
-  // When set, routed A rows are gathered on the fly: row p of a routed
-  // group is row gather_perm[p] / gather_k of map a_g (one-row boxes).
-  const int32_t* gather_perm;
-  int32_t gather_k;
 };
 
 // A maps: rank 2 {K, rows}; B maps: rank 3 {K, N rows, experts}; bf16, box
 // {64, 128 (A) or BN (B)}, 128-byte swizzle.
 struct GemmMaps {
   CUtensorMap a_r, a_s, b_r, b_s;
-  CUtensorMap a_g;  // token rows for gathered routed A tiles (box {64, 1})
 };
 
 bool make_map_bf16(CUtensorMap* map, int rank, const void* base, uint64_t inner, uint64_t rows,

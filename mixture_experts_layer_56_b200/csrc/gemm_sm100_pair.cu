@@ -105,8 +105,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
                          const __grid_constant__ CUtensorMap tmA_s,
                          const __grid_constant__ CUtensorMap tmB_r,
-                         const __grid_constant__ CUtensorMap tmB_s,
-                         const __grid_constant__ CUtensorMap tmA_g, const GroupedGemmArgs args) {
+                         const __grid_constant__ CUtensorMap tmB_s, const GroupedGemmArgs args) {
   constexpr int STAGES = pair_stages<BN, EPI>();
   constexpr uint32_t A_BYTES = HBM_ROWS * PBK * 2;
   constexpr uint32_t B_BYTES = (BN / 2) * PBK * 2;
@@ -208,9 +207,6 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
 
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer ----
-    // lane 0 owns the barriers and the tile loads; when routed A rows are
-    // gathered, every lane also issues one 4-row gather per k-block.  All
-    // bytes of both CTAs are counted on the leader's "full" barrier.
     if (lane == 0) {
       tma_prefetch_desc(&tmA_r);
       tma_prefetch_desc(&tmB_r);
@@ -218,47 +214,28 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         tma_prefetch_desc(&tmA_s);
         tma_prefetch_desc(&tmB_s);
       }
-      if (args.gather_perm) tma_prefetch_desc(&tmA_g);
-    }
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int tile = cluster; tile < total_tiles && ok; tile += nclusters) {
-      const PairTile ti =
-          decode_pair_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
-      const CUtensorMap* ma = ti.shared ? &tmA_s : &tmA_r;
-      const CUtensorMap* mb = ti.shared ? &tmB_s : &tmB_r;
-      const int my0 = ti.m_blk * PBM + static_cast<int>(rank) * HBM_ROWS;
-      const int row = grp_row0[ti.g] + my0;
-      const int nrow = ti.n_blk * BN + static_cast<int>(rank) * (BN / 2);
-      const int nkb = ti.shared ? args.kb_shared : args.kb_routed;
-      const int zbase = ti.shared ? 0 : ti.g - hs;
-      const bool gath = !ti.shared && args.gather_perm != nullptr;
-      int tok[4] = {0, 0, 0, 0};
-      if (gath) {
-        const int valid = grp_rows[ti.g] - my0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int rr = 4 * lane + j;
-          tok[j] = rr < valid ? args.gather_perm[row + rr] / args.gather_k : 0;
-        }
-      }
-      for (int kb = 0; kb < nkb; ++kb) {
-        int got = 1;
-        if (lane == 0) got = wait_bounded(empty_bar(stage), phase ^ 1u, abort_p, args.status) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, got, 0)) { ok = false; break; }
-        const uint32_t sa = smem_base + stage * STAGE_BYTES;
-        const uint32_t fb = leader ? full_bar(stage) : map_to_cta(full_bar(stage), 0);
-        if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < total_tiles && ok; tile += nclusters) {
+        const PairTile ti =
+            decode_pair_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+        const CUtensorMap* ma = ti.shared ? &tmA_s : &tmA_r;
+        const CUtensorMap* mb = ti.shared ? &tmB_s : &tmB_r;
+        const int row = grp_row0[ti.g] + ti.m_blk * PBM + static_cast<int>(rank) * HBM_ROWS;
+        const int nrow = ti.n_blk * BN + static_cast<int>(rank) * (BN / 2);
+        const int nkb = ti.shared ? args.kb_shared : args.kb_routed;
+        const int zbase = ti.shared ? 0 : ti.g - hs;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_p, args.status)) { ok = false; break; }
+          const uint32_t sa = smem_base + stage * STAGE_BYTES;
+          const uint32_t fb = leader ? full_bar(stage) : map_to_cta(full_bar(stage), 0);
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-          if (!gath) tma_load_2d_pair(sa, ma, fb, kb * PBK, row);
+          tma_load_2d_pair(sa, ma, fb, kb * PBK, row);
           tma_load_3d_pair(sa + A_BYTES, mb, fb, (kb % args.kb_per_expert) * PBK, nrow,
                            zbase + kb / args.kb_per_expert);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        __syncwarp();
-        if (gath)
-          tma_gather4_pair(sa + lane * 512, &tmA_g, fb, kb * PBK, tok[0], tok[1], tok[2], tok[3]);
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
     }
     __syncwarp();
@@ -421,7 +398,7 @@ int launch_pair_impl(const GemmMaps& m, const GroupedGemmArgs& args, int cluster
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, m.a_r, m.a_s, m.b_r, m.b_s, m.a_g, args) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kern, m.a_r, m.a_s, m.b_r, m.b_s, args) != cudaSuccess)
     return MOE_ERR_CUDA;
   count_launch();
   return check_launch();

@@ -182,6 +182,81 @@ dispatch_scatter_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n
   }
 }
 
+// The whole dispatch in one block, for batches of at most kDispatchChunk
+// tokens (decode): counts, the scan over experts and the scatter.
+template <int NW, int KMAX>
+__global__ void __launch_bounds__(kDispThreads)
+dispatch_single_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n,
+                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                       int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  __shared__ int wc[kDispWarps][256];
+  __shared__ int tot[256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = threadIdx.x;
+  int ek[KMAX];
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k) ek[k] = (t < T && k < K) ? idx[t * K + k] : -1;
+  uint32_t mask[NW];
+#pragma unroll
+  for (int w = 0; w < NW; ++w) mask[w] = 0;
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k)
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+      if (ek[k] >= 0 && (ek[k] >> 5) == w) mask[w] |= 1u << (ek[k] & 31);
+  warp_counts<NW>(mask, n, warp, lane, wc);
+  __syncthreads();
+  // per-expert totals (two experts per thread), then an exclusive scan
+  for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+    int c = 0;
+    if (e < n)
+      for (int w = 0; w < kDispWarps; ++w) c += wc[w][e];
+    tot[e] = c;
+    if (e < n) counts[e] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < n; ++e) {
+      const int c = tot[e];
+      tot[e] = run;
+      offsets[e] = run;
+      run += c;
+    }
+    offsets[n] = run;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    int run = tot[e];
+    for (int w = 0; w < kDispWarps; ++w) {
+      const int c = wc[w][e];
+      wc[w][e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    for (int b = 0; b < 32; ++b) {
+      const int e = w * 32 + b;
+      if (e >= n) break;
+      const bool has = (mask[w] >> b) & 1u;
+      const unsigned bal = __ballot_sync(kFull, has);
+      if (has) {
+        const int pos = wc[warp][e] + __popc(bal & lt);
+        int kk = 0;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k)
+          if (ek[k] == e) kk = k;
+        const int64_t slot = t * K + kk;
+        perm[pos] = static_cast<int32_t>(slot);
+        inv[slot] = pos;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // gather: xperm[p] = u[perm[p] / K]  (the rows each expert multiplies)
 // ---------------------------------------------------------------------------
@@ -225,50 +300,51 @@ __global__ void __launch_bounds__(256, 4)
 combine_kernel(const T* __restrict__ u, const float* __restrict__ ysh, const T* __restrict__ y,
                const float* __restrict__ w, const int32_t* __restrict__ inv, int64_t Tn, int d,
                int K, T* __restrict__ h) {
+  // one warp per (token, block of 32*V columns)
   constexpr int V = Vec16<T>::N;
   const int lane = threadIdx.x & 31;
+  const int nblk = (d + 32 * V - 1) / (32 * V);
+  const int64_t units = Tn * nblk;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       t < Tn; t += warps) {
-    // lane k < K holds row inv[t*K+k] and gate w[t*K+k]; shuffles hand them out
-    // y rows: inv[t*K+k] (expert order) or t*K+k (token-slot order, inv NULL)
+  for (int64_t wu = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       wu < units; wu += warps) {
+    const int64_t t = wu / nblk;
+    const int c = static_cast<int>(wu - t * nblk) * 32 * V + lane * V;
+    const bool live = c < d;
+    // lane k < K holds row inv[t*K+k] (or the token-slot row t*K+k) and
+    // gate w[t*K+k]; shuffles hand them to every lane
     const int my_row = lane < K ? (inv ? inv[t * K + lane] : static_cast<int>(t * K + lane)) : 0;
     const float my_w = lane < K ? w[t * K + lane] : 0.0f;
-    // the trip count is the same for every lane, so the shuffles stay converged
-    for (int c0 = 0; c0 < d; c0 += 32 * V) {
-      const int c = c0 + lane * V;
-      const bool live = c < d;
-      float acc[V], tmp[V];
-      if (live) {
-        Vec16<T>::load(u + t * d + c, acc);
+    float acc[V], tmp[V];
+    if (live) {
+      Vec16<T>::load(u + t * d + c, acc);
 #pragma unroll
-        for (int i = 0; i < V; i += 4) {
-          Vec16<float>::load(ysh + t * d + c + i, tmp);
+      for (int i = 0; i < V; i += 4) {
+        Vec16<float>::load(ysh + t * d + c + i, tmp);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i + j] += tmp[j];
-        }
+        for (int j = 0; j < 4; ++j) acc[i + j] += tmp[j];
       }
-      for (int k0 = 0; k0 < K; k0 += kCombineBatch) {
-        uint4 raw[kCombineBatch];
-        float wk[kCombineBatch];
-#pragma unroll
-        for (int kk = 0; kk < kCombineBatch; ++kk) {
-          const int k = k0 + kk;
-          const int64_t r = __shfl_sync(kFull, my_row, k & 31);
-          wk[kk] = __shfl_sync(kFull, my_w, k & 31);
-          if (live && k < K) raw[kk] = *reinterpret_cast<const uint4*>(y + r * d + c);
-        }
-#pragma unroll
-        for (int kk = 0; kk < kCombineBatch; ++kk) {
-          if (live && k0 + kk < K) {
-            Vec16<T>::load(reinterpret_cast<const T*>(&raw[kk]), tmp);
-#pragma unroll
-            for (int j = 0; j < V; ++j) acc[j] = fmaf(wk[kk], tmp[j], acc[j]);
-          }
-        }
-      }
-      if (live) Vec16<T>::store(h + t * d + c, acc);
     }
+    for (int k0 = 0; k0 < K; k0 += kCombineBatch) {
+      uint4 raw[kCombineBatch];
+      float wk[kCombineBatch];
+#pragma unroll
+      for (int kk = 0; kk < kCombineBatch; ++kk) {
+        const int k = k0 + kk;
+        const int64_t r = __shfl_sync(kFull, my_row, k & 31);
+        wk[kk] = __shfl_sync(kFull, my_w, k & 31);
+        if (live && k < K) raw[kk] = *reinterpret_cast<const uint4*>(y + r * d + c);
+      }
+#pragma unroll
+      for (int kk = 0; kk < kCombineBatch; ++kk) {
+        if (live && k0 + kk < K) {
+          Vec16<T>::load(reinterpret_cast<const T*>(&raw[kk]), tmp);
+#pragma unroll
+          for (int j = 0; j < V; ++j) acc[j] = fmaf(wk[kk], tmp[j], acc[j]);
+        }
+      }
+    }
+    if (live) Vec16<T>::store(h + t * d + c, acc);
   }
 }
 
@@ -451,6 +527,29 @@ int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_
       return MOE_ERR_CUDA;
     return MOE_OK;
   }
+  if (nch == 1) {
+    // one block does it all
+#define MOE_SINGLE_CASE(W)                                                                   \
+  case W:                                                                                    \
+    if (K <= 8)                                                                              \
+      dispatch_single_kernel<W, 8><<<1, kDispThreads, 0, st>>>(idx, T, K, n, counts, offsets,  \
+                                                               perm, inv);                   \
+    else if (K <= 16)                                                                        \
+      dispatch_single_kernel<W, 16><<<1, kDispThreads, 0, st>>>(idx, T, K, n, counts, offsets, \
+                                                                perm, inv);                  \
+    else                                                                                     \
+      dispatch_single_kernel<W, 32><<<1, kDispThreads, 0, st>>>(idx, T, K, n, counts, offsets, \
+                                                                perm, inv);                  \
+    break;
+    switch (nw) {
+      MOE_SINGLE_CASE(1) MOE_SINGLE_CASE(2) MOE_SINGLE_CASE(3) MOE_SINGLE_CASE(4)
+      MOE_SINGLE_CASE(5) MOE_SINGLE_CASE(6) MOE_SINGLE_CASE(7) MOE_SINGLE_CASE(8)
+      default: return MOE_ERR_SHAPE;
+    }
+#undef MOE_SINGLE_CASE
+    count_launch();
+    return check_launch();
+  }
 #define MOE_DISPATCH_CASE(W)                                                                 \
   case W:                                                                                    \
     dispatch_count_kernel<W><<<static_cast<unsigned>(nch), kDispThreads, 0, st>>>(idx, T, K, n, \
@@ -506,7 +605,8 @@ int launch_gather(int dtype, const void* u, const int32_t* perm, int64_t rows, i
 int launch_combine(int dtype, const void* u, const float* ysh, const void* y, const float* w,
                    const int32_t* inv, int64_t T, int d, int K, void* h, cudaStream_t st) {
   if (T == 0) return MOE_OK;
-  const unsigned grid = grid_for_rows(T, 8);
+  const int V = dtype == MOE_DTYPE_BF16 ? 8 : 4;
+  const unsigned grid = grid_for_rows(T * ((d + 32 * V - 1) / (32 * V)), 8);
   if (dtype == MOE_DTYPE_BF16)
     combine_kernel<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16*>(u), ysh,
                                                static_cast<const bf16*>(y), w, inv, T, d, K,

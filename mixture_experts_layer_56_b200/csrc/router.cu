@@ -61,7 +61,7 @@ __device__ __forceinline__ uint4 lds_sw128(const uint8_t* tile, int row, int ch)
   return *reinterpret_cast<const uint4*>(tile + row * 128 + ((ch ^ (row & 7)) << 4));
 }
 
-template <typename TIn, int EPT, bool STATS>
+template <typename TIn, int EPT, bool STATS, int CS>
 __global__ void __launch_bounds__(kRouterThreads)
 router_topk_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmE,
                    const float* __restrict__ bias, int64_t T, int d, int n, int K, int flags,
@@ -89,8 +89,12 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constan
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTokPerCta;
-  const int nchunks = (d + KC - 1) / KC;
+  // a cluster of CS CTAs shares 32 tokens; CTA `rank` sums its share of d
+  const uint32_t rank = CS > 1 ? cluster_ctarank() : 0;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x / CS) * kTokPerCta;
+  const int nall = (d + KC - 1) / KC;
+  const int cbeg = static_cast<int>(rank) * nall / CS;
+  const int nchunks = (static_cast<int>(rank) + 1) * nall / CS - cbeg;
   volatile int* abort_p = &abort_flag;
 
   if (tid == 0) {
@@ -121,8 +125,8 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constan
         if (!wait_bounded(empty_bar(st), ph ^ 1u, abort_p, nullptr)) break;
         const uint32_t sb = ring_base + st * ST_BYTES;
         mbar_arrive_expect_tx(full_bar(st), ST_BYTES);
-        tma_load_2d(sb, &tmU, full_bar(st), c * KC, static_cast<int32_t>(t0));
-        tma_load_2d(sb + U_BYTES, &tmE, full_bar(st), c * KC, 0);
+        tma_load_2d(sb, &tmU, full_bar(st), (cbeg + c) * KC, static_cast<int32_t>(t0));
+        tma_load_2d(sb + U_BYTES, &tmE, full_bar(st), (cbeg + c) * KC, 0);
       }
     }
     __syncwarp();
@@ -187,6 +191,22 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constan
       }
   }
   __syncthreads();
+  if (CS > 1) {
+    // rank 0 adds the other CTAs' partial logits, in rank order, through
+    // distributed shared memory
+    cluster_sync_all();
+    if (rank == 0) {
+      const uint32_t base = smem_addr(sL);
+      for (int i = tid; i < kTokPerCta * LDL; i += blockDim.x) {
+        float a = sL[i];
+        for (int r = 1; r < CS; ++r) a += ld_shared_cluster_f32(map_to_cta(base + 4u * i, r));
+        sL[i] = a;
+      }
+    }
+    cluster_sync_all();  // the peers' logits stay alive until read
+    if (rank != 0) return;
+    __syncthreads();
+  }
 
   float b[EPT];
 #pragma unroll
@@ -284,7 +304,7 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constan
     for (int e = threadIdx.x; e < n; e += blockDim.x) {
       float a = 0.0f;
       for (int ww = 0; ww < kRouterWarps; ++ww) a += pred[ww * NP + e];
-      pstat[static_cast<int64_t>(blockIdx.x) * n + e] = a;
+      pstat[static_cast<int64_t>(blockIdx.x / CS) * n + e] = a;
     }
   }
 }
@@ -304,16 +324,39 @@ int launch_router_t(const TIn* u, const TIn* E, const float* bias, int64_t T, in
       !make_map_2d(&me, dt, E, static_cast<uint64_t>(d), static_cast<uint64_t>(n),
                    static_cast<uint64_t>(d) * sizeof(TIn), 8 * VPC, 32 * ept))
     return MOE_ERR_CUDA;
+  // small batches: split d over a cluster of CS CTAs so that more SMs work
+  const int nall = static_cast<int>((d + 8 * VPC - 1) / (8 * VPC));
+  int cs = 1;
+  while (cs < 8 && static_cast<int64_t>(grid) * cs * 2 <= 148 && cs * 2 <= nall) cs *= 2;
+  auto launch = [&](auto kern, int smem) -> int {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid * cs, 1, 1);
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mu, me, bias, T, d, n, K, flags, idx, w, pstat) ==
+                   cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+  };
+  int rc = MOE_OK;
 #define MOE_ROUTER_CASE(N)                                                                  \
-  case N: {                                                                                 \
-    auto kern = router_topk_kernel<TIn, N, STATS>;                                          \
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,             \
-                             router_smem_bytes<N>()) != cudaSuccess)                        \
-      return MOE_ERR_CUDA;                                                                  \
-    kern<<<grid, block, router_smem_bytes<N>(), st>>>(mu, me, bias, T, d, n, K, flags, idx, w, \
-                                                     pstat);                                \
-    break;                                                                                  \
-  }
+  case N:                                                                                   \
+    rc = cs == 8   ? launch(router_topk_kernel<TIn, N, STATS, 8>, router_smem_bytes<N>())    \
+         : cs == 4 ? launch(router_topk_kernel<TIn, N, STATS, 4>, router_smem_bytes<N>())    \
+         : cs == 2 ? launch(router_topk_kernel<TIn, N, STATS, 2>, router_smem_bytes<N>())    \
+                   : launch(router_topk_kernel<TIn, N, STATS, 1>, router_smem_bytes<N>());   \
+    break;
   switch (ept) {
     MOE_ROUTER_CASE(1)
     MOE_ROUTER_CASE(2)
@@ -327,6 +370,7 @@ int launch_router_t(const TIn* u, const TIn* E, const float* bias, int64_t T, in
       return MOE_ERR_SHAPE;
   }
 #undef MOE_ROUTER_CASE
+  if (rc) return rc;
   count_launch();
   return check_launch();
 }

@@ -39,9 +39,7 @@ def test_tiny_fp32_config_full():
     print(rep["near_ties"], rep["err_h"])
 
 
-GEMM_MODES = {"single_cta": L.MOE_FLAG_GEMM_SINGLE_CTA, "cta_pair": L.MOE_FLAG_GEMM_CTA_PAIR,
-              "single_cta_tma_gather": L.MOE_FLAG_GEMM_SINGLE_CTA | L.MOE_FLAG_GEMM_TMA_GATHER,
-              "cta_pair_tma_gather": L.MOE_FLAG_GEMM_CTA_PAIR | L.MOE_FLAG_GEMM_TMA_GATHER}
+GEMM_MODES = {"single_cta": L.MOE_FLAG_GEMM_SINGLE_CTA, "cta_pair": L.MOE_FLAG_GEMM_CTA_PAIR}
 
 
 @pytest.mark.parametrize("mode", sorted(GEMM_MODES))
