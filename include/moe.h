@@ -63,6 +63,7 @@ enum {
   MOE_ERR_CUDA = -6,         /* CUDA runtime / launch error */
   MOE_ERR_DEVICE_CHECK = -7, /* a kernel gave up waiting (see moe_read_status) */
   MOE_ERR_UNSUPPORTED = -8,  /* no device of compute capability 10.0 */
+  MOE_ERR_SCRATCH_LIMIT = -9, /* shape too large for moe_dispatch_static_scratch */
 };
 
 /* Router flags (moe_shape_t.flags). */
@@ -127,6 +128,28 @@ int moe_route(const moe_shape_t* shape, const void* u, const void* E,
 int moe_dispatch(const moe_shape_t* shape, const int32_t* idx, int32_t* counts,
                  int32_t* offsets, int32_t* perm, int32_t* inv, void* ws,
                  size_t ws_bytes, moe_stream_t stream);
+
+/* The same dispatch as moe_dispatch, same outputs bit for bit, for callers
+   that cannot supply device memory per call: the paper has no counterpart;
+   it is an interface for embedders.  Allocation may synchronise the device
+   or fail once a caching pool holds the GPU's memory, so a latency-bound
+   serving loop, or a host library without an allocator of its own, may not
+   be able to provide `ws`.  This call allocates nothing: its scratch is one
+   fixed array of MOE_DISPATCH_STATIC_SCRATCH_BYTES inside libmoe.
+   Limit: 2 * round_up_256(ceil(T/128) * n_routed * 4) bytes must fit in
+   that array (T <= 32768 at 256 routed experts, T <= 131072 at 64);
+   larger shapes return MOE_ERR_SCRATCH_LIMIT before any launch.
+   Set-up: the first call on each device (current device at the call)
+   looks up the array's device address; make that first call before any
+   stream capture begins on the device.
+   Sharing: every call in the process, on any stream, uses the same array.
+   Calls whose kernels may overlap on a device race on it and corrupt each
+   other's perm/inv/offsets; order them (one stream, or events).  Nothing in
+   the array has to start at zero: each call writes every entry it reads. */
+#define MOE_DISPATCH_STATIC_SCRATCH_BYTES (512u * 1024u)
+int moe_dispatch_static_scratch(const moe_shape_t* shape, const int32_t* idx,
+                                int32_t* counts, int32_t* offsets, int32_t* perm,
+                                int32_t* inv, moe_stream_t stream);
 
 /* a4-a6, expert FFNs: for every position p of expert e's segment,
    y[p] = FFN_e(u_{perm[p]/top_k}); and ysh[t] = sum_s FFN_s(u_t) over the

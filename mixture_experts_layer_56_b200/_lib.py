@@ -29,6 +29,8 @@ MOE_ERR_DTYPE = -5
 MOE_ERR_CUDA = -6
 MOE_ERR_DEVICE_CHECK = -7
 MOE_ERR_UNSUPPORTED = -8
+MOE_ERR_SCRATCH_LIMIT = -9
+MOE_DISPATCH_STATIC_SCRATCH_BYTES = 512 * 1024
 
 
 class MoeError(RuntimeError):
@@ -60,6 +62,7 @@ SIGNATURES = {
     "moe_pack_w13": (c_int, [_SHAPE, c_int32, _V, _V, _V, _V]),
     "moe_route": (c_int, [_SHAPE, _V, _V, _V, _V, _V, _V]),
     "moe_dispatch": (c_int, [_SHAPE, _V, _V, _V, _V, _V, _V, c_size_t, _V]),
+    "moe_dispatch_static_scratch": (c_int, [_SHAPE, _V, _V, _V, _V, _V, _V]),
     "moe_expert_ffn": (c_int, [_SHAPE, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, c_size_t, _V]),
     "moe_combine": (c_int, [_SHAPE, _V, _V, _V, _V, _V, _V, _V]),
     "moe_layer_forward": (c_int, [_SHAPE, _V, _V, _V, _V, _V, _V, _V, _V, _V, c_size_t, _V]),
@@ -159,6 +162,12 @@ def moe_dispatch(shape, idx, counts, offsets, perm, inv, ws, ws_bytes=None, stre
     return _check("moe_dispatch", lib().moe_dispatch(
         ctypes.byref(shape), _ptr(idx), _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
         _ptr(ws), nb, _stream(stream)))
+
+
+def moe_dispatch_static_scratch(shape, idx, counts, offsets, perm, inv, stream=None):
+    return _check("moe_dispatch_static_scratch", lib().moe_dispatch_static_scratch(
+        ctypes.byref(shape), _ptr(idx), _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv),
+        _stream(stream)))
 
 
 def moe_expert_ffn(shape, u, perm, offsets, W13, W2, W13_s, W2_s, y, ysh, ws, ws_bytes=None,

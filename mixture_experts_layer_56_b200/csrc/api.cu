@@ -369,6 +369,7 @@ const char* moe_strerror(int status) {
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_DEVICE_CHECK: return "a kernel gave up waiting (device check)";
     case MOE_ERR_UNSUPPORTED: return "device is not sm_100 (B200)";
+    case MOE_ERR_SCRATCH_LIMIT: return "shape exceeds the fixed dispatch scratch";
     default: return "unknown status";
   }
 }
