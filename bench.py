@@ -295,6 +295,10 @@ def run_ours(args):
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier()
     launches0 = L.moe_launch_count()
+    # per-stage CUDA events on the launching stream, inside the timed steps
+    # (graph replays carry no events: those are timed in a separate pass)
+    L.moe_profile_read()
+    L.moe_profile_enable(graph is None)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         for i in range(args.steps):
             flush.zero_()
@@ -303,6 +307,8 @@ def run_ours(args):
             ends[i].record(stream)
         barrier()
     launches = L.moe_launch_count() - launches0
+    recs = L.moe_profile_read()
+    L.moe_profile_enable(False)
     if graph is not None:
         # replays bypass the library's launch counter: count one eager step
         c0 = L.moe_launch_count()
@@ -317,15 +323,15 @@ def run_ours(args):
     ms_per_step = total_ms / args.steps
     tflops = wl.expert_flops() * world * args.steps / (total_ms / 1e3) / 1e12
 
-    # ---- per-kernel device time (events around each stage), untimed pass --
-    L.moe_profile_enable(True)
-    prof_steps = 5
-    for _ in range(prof_steps):
-        flush.zero_()
-        forward()
-    torch.cuda.synchronize(dev)
-    recs = L.moe_profile_read()
-    L.moe_profile_enable(False)
+    if graph is not None:
+        # ---- per-kernel device time for the graph run: an eager pass --------
+        L.moe_profile_enable(True)
+        for _ in range(5):
+            flush.zero_()
+            forward()
+        torch.cuda.synchronize(dev)
+        recs = L.moe_profile_read()
+        L.moe_profile_enable(False)
     per_kernel = {}
     for name, ms in recs:
         per_kernel.setdefault(name, []).append(ms)
