@@ -80,6 +80,13 @@ enum {
      same up to fp32 summation order inside the tensor cores. */
   MOE_FLAG_GEMM_SINGLE_CTA = 2,
   MOE_FLAG_GEMM_CTA_PAIR = 4,
+  /* bf16 router on the CUDA cores: each logit is two fp32 FMA chains over
+     the halves of d in increasing j, added once.  Default (0): the logits
+     are one tcgen05 MMA tile per 128 tokens (bf16 products are exact in
+     fp32; fp32 accumulation in the tensor cores' own order).  The two agree
+     up to fp32 summation order.  The fp32 dtype always uses the CUDA
+     cores. */
+  MOE_FLAG_ROUTER_SIMT = 8,
 };
 
 /* Layer shape.  Limits: 1 <= n_routed <= 256, 1 <= top_k <= min(n_routed, 32),
@@ -112,7 +119,8 @@ int moe_pack_w13(const moe_shape_t* shape, int32_t n_experts, const void* W1,
                  const void* W3, void* W13, moe_stream_t stream);
 
 /* a1-a2, router (eqs. (10)-(11)): logits u_t.e_i (+ b_i) accumulated in fp32
-   in order j = 0..d-1, softmax over the n_routed experts, top-K.
+   (tensor cores for bf16, see MOE_FLAG_ROUTER_SIMT), softmax over the
+   n_routed experts, top-K.
    u: [T, d]; E: [n_routed, d]; bias: [n_routed] float32 or NULL.
    Outputs idx: [T, top_k] int32 in descending score order (ties: lower
    index first); w: [T, top_k] float32 gates (not renormalised). */
@@ -212,8 +220,11 @@ int moe_read_status(const void* ws, int32_t* status, moe_stream_t stream);
    for those events and returns, oldest first, the stage kind (MOE_KERNEL_*)
    and elapsed milliseconds of each bracketed launch since the last read:
    at most `max` entries are written and *count receives the number
-   written; up to 4096 are kept, later ones are dropped.  Enabling adds event
-   records between launches and never changes any result. */
+   written; up to 4096 are kept, later ones are dropped.  `on`: 0 = off,
+   1 = every stage, otherwise a mask of (1 << MOE_KERNEL_*) bits naming the
+   stages to bracket (each bracket adds two event records to the stream, so
+   a mask keeps the timing of the other stages undisturbed).  Tracing never
+   changes any result. */
 enum {
   MOE_KERNEL_ROUTER = 1,
   MOE_KERNEL_DISPATCH = 2,

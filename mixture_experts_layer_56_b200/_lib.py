@@ -19,6 +19,7 @@ MOE_DTYPE_BF16 = 1
 MOE_FLAG_BIAS_SELECT_ONLY = 1
 MOE_FLAG_GEMM_SINGLE_CTA = 2
 MOE_FLAG_GEMM_CTA_PAIR = 4
+MOE_FLAG_ROUTER_SIMT = 8
 
 MOE_OK = 0
 MOE_ERR_NULLPTR = -1
@@ -30,6 +31,15 @@ MOE_ERR_CUDA = -6
 MOE_ERR_DEVICE_CHECK = -7
 MOE_ERR_UNSUPPORTED = -8
 MOE_ERR_SCRATCH_LIMIT = -9
+
+# stage kinds of the tracer (include/moe.h MOE_KERNEL_*)
+MOE_KERNEL_ROUTER = 1
+MOE_KERNEL_DISPATCH = 2
+MOE_KERNEL_GATHER = 3
+MOE_KERNEL_GEMM_GATE_UP = 4
+MOE_KERNEL_GEMM_DOWN = 5
+MOE_KERNEL_COMBINE = 6
+MOE_KERNEL_FFN_F32 = 7
 MOE_DISPATCH_STATIC_SCRATCH_BYTES = 512 * 1024
 
 
@@ -213,8 +223,18 @@ def moe_read_status(ws, stream=None) -> int:
     return st.value
 
 
-def moe_profile_enable(on: bool = True):
-    return _check("moe_profile_enable", lib().moe_profile_enable(1 if on else 0))
+def moe_profile_enable(on=True, kinds=None):
+    """Turn stage tracing on or off; `kinds` (MOE_KERNEL_* values) limits it
+    to those stages."""
+    if not on:
+        v = 0
+    elif kinds is None:
+        v = 1
+    else:
+        v = 0
+        for k in kinds:
+            v |= 1 << int(k)
+    return _check("moe_profile_enable", lib().moe_profile_enable(v))
 
 
 def moe_profile_read(max_entries: int = 4096):

@@ -29,6 +29,7 @@ struct ProfRec {
 struct Profiler {
   std::mutex mu;
   std::atomic<bool> on{false};
+  std::atomic<uint32_t> mask{~0u};  // bit k: bracket stages of kind k
   std::vector<ProfRec> recs;
   std::vector<cudaEvent_t> pool;
   cudaEvent_t get() {
@@ -54,7 +55,7 @@ class Stage {
  public:
   Stage(int32_t kind, cudaStream_t st) : st_(st) {
     Profiler& p = prof();
-    if (!p.on.load()) return;
+    if (!p.on.load() || kind < 0 || kind > 31 || !((p.mask.load() >> kind) & 1u)) return;
     std::lock_guard<std::mutex> lock(p.mu);
     if (p.recs.size() >= kMaxProfRecs) return;
     ProfRec r{kind, p.get(), p.get()};
@@ -131,7 +132,7 @@ int validate(const moe_shape_t* s) {
       s->inter < 1)
     return MOE_ERR_SHAPE;
   const int32_t known = MOE_FLAG_BIAS_SELECT_ONLY | MOE_FLAG_GEMM_SINGLE_CTA |
-                        MOE_FLAG_GEMM_CTA_PAIR;
+                        MOE_FLAG_GEMM_CTA_PAIR | MOE_FLAG_ROUTER_SIMT;
   if ((s->flags & ~known) != 0) return MOE_ERR_SHAPE;
   if ((s->flags & MOE_FLAG_GEMM_SINGLE_CTA) && (s->flags & MOE_FLAG_GEMM_CTA_PAIR))
     return MOE_ERR_SHAPE;
@@ -328,7 +329,8 @@ int forward_device(const moe_shape_t& s, const Layout& L, const void* u, const v
   float* ysh = at<float>(ws, L.ysh);
   {
     Stage sg(MOE_KERNEL_ROUTER, st);
-    if (int rc = launch_router(s.dtype, u, E, bias, T, s.d, n, K, s.flags, idx, w, nullptr, st))
+    if (int rc = launch_router(s.dtype, u, E, bias, T, s.d, n, K, s.flags, idx, w, nullptr,
+                               at<int32_t>(ws, L.status), st))
       return rc;
   }
   {
@@ -379,6 +381,7 @@ const char* moe_version(void) { return "moe-b200 0.1.0 (sm_100a)"; }
 uint64_t moe_launch_count(void) { return g_launches.load(); }
 
 int moe_profile_enable(int on) {
+  prof().mask.store(on == 1 ? ~0u : static_cast<uint32_t>(on));
   prof().on.store(on != 0);
   return MOE_OK;
 }
@@ -463,7 +466,7 @@ int moe_route(const moe_shape_t* shape, const void* u, const void* E, const floa
   if (int rc = device_info(&di)) return rc;
   Stage sg(MOE_KERNEL_ROUTER, static_cast<cudaStream_t>(stream));
   return launch_router(shape->dtype, u, E, bias, shape->T, shape->d, shape->n_routed,
-                       shape->top_k, shape->flags, idx, w, nullptr,
+                       shape->top_k, shape->flags, idx, w, nullptr, nullptr,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -586,7 +589,7 @@ int moe_expert_balance(const moe_shape_t* shape, const void* u, const void* E, c
   // the router pass also rewrites the workspace's idx / w scratch
   if (int rc = launch_router(shape->dtype, u, E, bias, shape->T, shape->d, shape->n_routed,
                              shape->top_k, shape->flags, at<int32_t>(ws, L.idx), at<float>(ws, L.w),
-                             pstat, st))
+                             pstat, at<int32_t>(ws, L.status), st))
     return rc;
   return launch_balance_reduce(pstat, router_num_ctas(shape->T), counts, shape->T,
                                shape->n_routed, shape->top_k, f, P, st);

@@ -209,6 +209,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
             int dummy = 0;
             wait_bounded(full_bar(s), (issued_parity >> s) & 1u, &dummy, nullptr);
           }
+      } else {
+        // the last round's "empty" arrivals land in this CTA's shared memory:
+        // wait for them so that none is still in flight when the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) {
+            int dummy = 0;
+            wait_bounded(empty_bar(s), (issued_parity >> s) & 1u, &dummy, nullptr);
+          }
       }
     }
     __syncwarp();

@@ -38,7 +38,7 @@ constexpr int kStageRowBytes = 128;
 constexpr int kStagePitch = kStageRowBytes + 16;
 constexpr int kWarpStageBytes = 32 * kStagePitch;
 
-template <int EPI> constexpr int pair_epi_warps() { return EPI == kEpiSwiGLU ? 8 : 4; }
+template <int EPI> constexpr int pair_epi_warps() { return 8; }
 
 // pipeline depth: as many 256-row k-block stages as fit beside the staging
 template <int BN, int EPI>
@@ -112,8 +112,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr uint32_t IDESC = idesc_bf16_f32(PBM, BN);
-  // SwiGLU epilogues drain with 8 warps (two per TMEM lane quarter, one per
-  // half of the columns); plain ones with 4
+  // epilogues drain with 8 warps: two per TMEM lane quarter, one per half
+  // of the tile's columns
   constexpr int EPI_WARPS = pair_epi_warps<EPI>();
   constexpr uint16_t kBoth = 0x3;
 
@@ -215,7 +215,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         tma_prefetch_desc(&tmB_s);
       }
       int stage = 0;
-      uint32_t phase = 0;
+      uint32_t phase = 0, issued = 0, issued_parity = 0;
       bool ok = true;
       for (int tile = cluster; tile < total_tiles && ok; tile += nclusters) {
         const PairTile ti =
@@ -234,8 +234,19 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
           tma_load_2d_pair(sa, ma, fb, kb * PBK, row);
           tma_load_3d_pair(sa + A_BYTES, mb, fb, (kb % args.kb_per_expert) * PBK, nrow,
                            zbase + kb / args.kb_per_expert);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+      }
+      if (ok) {
+        // the last round's "empty" arrivals land in this CTA's shared memory:
+        // wait for them so that none is still in flight when the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) {
+            int dummy = 0;
+            wait_bounded(empty_bar(s), (issued_parity >> s) & 1u, &dummy, nullptr);
+          }
       }
     }
     __syncwarp();
@@ -331,33 +342,61 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
         }
         uint8_t* dst = live ? reinterpret_cast<uint8_t*>(out + orow * ld + col0) : nullptr;
         warp_store_rows<OC * 2>(stage, packed, dst, lane);
-      } else {
+      } else if (ti.shared) {
+        // fp32 shared-expert output: chunks of 32 columns (128 bytes a row);
+        // the TMEM load of chunk c+1 is in flight while chunk c is stored
+        constexpr int WC = BN / 2;
+        constexpr int NCH = WC / 32;
+        const int c0 = hcol * WC;
+        float x[32];
+        tmem_ld32(taddr + c0, x);
+        tmem_ld_wait_regs(x);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          float x[32];
-          tmem_ld32(taddr + c * 32, x);
-          tmem_ld_wait();
-          const int64_t col = static_cast<int64_t>(ti.n_blk) * BN + c * 32;
-          if (ti.shared) {
-            // fp32: 32 columns = 128 bytes per row
-            uint4 packed[8];
+        for (int c = 0; c < NCH; ++c) {
+          uint4 packed[8];
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              packed[v] = make_uint4(__float_as_uint(x[4 * v]), __float_as_uint(x[4 * v + 1]),
-                                     __float_as_uint(x[4 * v + 2]), __float_as_uint(x[4 * v + 3]));
-            uint8_t* dst = live ? reinterpret_cast<uint8_t*>(static_cast<float*>(args.out_s) +
-                                                             orow * args.ld_s + col)
-                                : nullptr;
-            warp_store_rows<128>(stage, packed, dst, lane);
-          } else {
-            // bf16: 32 columns = 64 bytes per row
-            uint4 packed[4];
+          for (int v = 0; v < 8; ++v)
+            packed[v] = make_uint4(__float_as_uint(x[4 * v]), __float_as_uint(x[4 * v + 1]),
+                                   __float_as_uint(x[4 * v + 2]), __float_as_uint(x[4 * v + 3]));
+          if (c + 1 < NCH) tmem_ld32(taddr + c0 + (c + 1) * 32, x);
+          const int64_t col = static_cast<int64_t>(ti.n_blk) * BN + c0 + c * 32;
+          uint8_t* dst = live ? reinterpret_cast<uint8_t*>(static_cast<float*>(args.out_s) +
+                                                           orow * args.ld_s + col)
+                              : nullptr;
+          warp_store_rows<128>(stage, packed, dst, lane);
+          if (c + 1 < NCH) tmem_ld_wait_regs(x);
+        }
+      } else {
+        // bf16 routed output: chunks of up to 64 columns (128 bytes a row),
+        // next chunk's TMEM load overlapping this chunk's stores
+        constexpr int WC = BN / 2;
+        constexpr int CW = WC < 64 ? WC : 64;
+        constexpr int NCH = WC / CW;
+        const int c0 = hcol * WC;
+        float x[CW];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) Vec16<bf16>::store(reinterpret_cast<bf16*>(&packed[v]), x + v * 8);
-            uint8_t* dst = live ? reinterpret_cast<uint8_t*>(static_cast<bf16*>(args.out_r) +
-                                                             prow * args.ld_r + col)
-                                : nullptr;
-            warp_store_rows<64>(stage, packed, dst, lane);
+        for (int h = 0; h < CW / 32; ++h) tmem_ld32(taddr + c0 + h * 32, x + h * 32);
+#pragma unroll
+        for (int h = 0; h < CW / 32; ++h) tmem_ld_wait_regs(x + h * 32);
+#pragma unroll 1
+        for (int c = 0; c < NCH; ++c) {
+          uint4 packed[CW / 8];
+#pragma unroll
+          for (int v = 0; v < CW / 8; ++v)
+            Vec16<bf16>::store(reinterpret_cast<bf16*>(&packed[v]), x + v * 8);
+          if (c + 1 < NCH) {
+#pragma unroll
+            for (int h = 0; h < CW / 32; ++h)
+              tmem_ld32(taddr + c0 + (c + 1) * CW + h * 32, x + h * 32);
+          }
+          const int64_t col = static_cast<int64_t>(ti.n_blk) * BN + c0 + c * CW;
+          uint8_t* dst = live ? reinterpret_cast<uint8_t*>(static_cast<bf16*>(args.out_r) +
+                                                           prow * args.ld_r + col)
+                              : nullptr;
+          warp_store_rows<CW * 2>(stage, packed, dst, lane);
+          if (c + 1 < NCH) {
+#pragma unroll
+            for (int h = 0; h < CW / 32; ++h) tmem_ld_wait_regs(x + h * 32);
           }
         }
       }

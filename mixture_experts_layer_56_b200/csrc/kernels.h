@@ -13,7 +13,12 @@ int router_num_ctas(int64_t T);
 
 int launch_router(int dtype, const void* u, const void* E, const float* bias, int64_t T, int d,
                   int n, int K, int flags, int32_t* idx, float* w, float* pstat,
-                  cudaStream_t st);
+                  int32_t* status, cudaStream_t st);
+
+// bf16 router on the tensor cores (router_tc.cu); pstat as launch_router's
+int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T, int d, int n,
+                     int K, int flags, int32_t* idx, float* w, float* pstat, int32_t* status,
+                     cudaStream_t st);
 
 int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_counts,
                     int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* perm,

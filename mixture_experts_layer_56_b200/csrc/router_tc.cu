@@ -1,0 +1,395 @@
+// Router of the DeepSeekMoE layer (§3.2, eqs. (10)-(11)) on the tensor
+// cores: the logits l_{t,i} = u_t . e_i of 128 tokens against every routed
+// expert are one tcgen05 MMA tile (M = 128 tokens, N = N_r rounded up to 16,
+// K = d), bf16 x bf16 with fp32 accumulation in TMEM.  Each product of two
+// bf16 values is exact in fp32, so the logits differ from a sequential fp32
+// sum only in summation order.
+//
+// One CTA per 128 tokens, 4 warps.  Warp 0 streams 64-wide column slices
+// of u (128 rows) and E (N rows, zero rows past N_r) into a shared-memory
+// ring with TMA; warp 1 issues the MMAs; warp 2 owns the TMEM columns.
+// Then every thread takes the token of its TMEM lane and works through its
+// logits in 32-column chunks read from TMEM:
+//   max and sum of the softmax (bias added unless it only steers the
+//   selection), then K selection passes, each taking the largest key
+//   l + b that comes after the previous pick in (value descending, index
+//   ascending) order, so lower indices win ties.  Gates are
+//   exp(l - max) / sum, not renormalised over the top K.
+// With statistics on, each warp also sums the scores of its 32 tokens per
+// expert (fixed token order) for the balance statistics of §3.3.
+#include <cuda.h>
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "gemm_sm100.h"
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kRtTokens = 128;  // tokens per CTA: one TMEM lane each
+constexpr int kRtThreads = 128;
+constexpr int kRtBK = 64;  // columns of d per stage (128 bytes of bf16)
+constexpr int kRtMaxStages = 8;
+constexpr int kRtSmemBudget = 200 * 1024;
+constexpr int kRtTileBytes = kRtTokens * kRtBK * 2;
+
+inline int rt_padded_experts(int n) { return (n + 15) / 16 * 16; }
+inline int rt_stage_bytes(int np) { return kRtTileBytes + np * kRtBK * 2; }
+inline int rt_stages(int np) {
+  const int s = kRtSmemBudget / rt_stage_bytes(np);
+  return s > kRtMaxStages ? kRtMaxStages : s;
+}
+
+// NCH > 0: a token's logits (NCH chunks of 32) stay in registers after one
+// TMEM read, SEL = the bias only steers the selection.  NCH = 0: any expert
+// count; the chunks are re-read from TMEM for every pass.
+template <bool STATS, int NCH, bool SEL>
+__global__ void __launch_bounds__(kRtThreads, 1)
+router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmE,
+                 const float* __restrict__ bias, int64_t T, int d, int n, int np, int K,
+                 int flags, int stages, uint32_t tmem_cols, int32_t* __restrict__ idx,
+                 float* __restrict__ w, float* __restrict__ pstat, int32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[2 * kRtMaxStages + 2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  __shared__ float sbias[256];
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t smem_base = smem_addr(smem);
+  const uint32_t stage_bytes = static_cast<uint32_t>(kRtTileBytes + np * kRtBK * 2);
+  const uint32_t bar_base = smem_addr(bars);
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (kRtMaxStages + s); };
+  const uint32_t done_bar = bar_base + 8u * (2 * kRtMaxStages);
+  const uint32_t drain_bar = bar_base + 8u * (2 * kRtMaxStages + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int m0 = static_cast<int>(blockIdx.x) * kRtTokens;
+  const int nkb = d / kRtBK;
+  volatile int* abort_p = &abort_flag;
+
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(done_bar, 1);
+    mbar_init(drain_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    fence_async_shared();
+  }
+  for (int e = tid; e < 256; e += kRtThreads) sbias[e] = (bias != nullptr && e < n) ? bias[e] : 0.0f;
+  if (warp == 2) {
+    tmem_alloc(smem_addr(&tmem_slot), tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  const uint32_t idesc = idesc_bf16_f32(kRtTokens, np);
+
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer ----
+    if (lane == 0) {
+      tma_prefetch_desc(&tmU);
+      tma_prefetch_desc(&tmE);
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_p, status)) { ok = false; break; }
+        const uint32_t sa = smem_base + stage * stage_bytes;
+        mbar_arrive_expect_tx(full_bar(stage), stage_bytes);
+        tma_load_2d(sa, &tmU, full_bar(stage), kb * kRtBK, m0);
+        tma_load_2d(sa + kRtTileBytes, &tmE, full_bar(stage), kb * kRtBK, 0);
+        issued |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == stages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) {
+        for (int s = 0; s < stages; ++s)
+          if (issued & (1u << s)) {
+            int dummy = 0;
+            wait_bounded(full_bar(s), (issued_parity >> s) & 1u, &dummy, nullptr);
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer ----
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!wait_bounded(full_bar(stage), phase, abort_p, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_base + stage * stage_bytes;
+        const uint32_t sb = sa + kRtTileBytes;
+#pragma unroll
+        for (int k = 0; k < kRtBK / 16; ++k)
+          mma_bf16(tmem_base, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32), idesc,
+                   (kb > 0 || k > 0) ? 1u : 0u);
+        // only stages that are loaded again need an "empty" arrival; the
+        // last round's would otherwise still be in flight when the CTA exits
+        if (kb + stages < nkb) mma_commit(empty_bar(stage));
+        if (++stage == stages) { stage = 0; phase ^= 1u; }
+      }
+      if (ok) {
+        mma_commit(done_bar);
+      } else {
+        mma_commit(drain_bar);
+        int dummy = 0;
+        wait_bounded(drain_bar, 0, &dummy, nullptr);
+      }
+    }
+    __syncwarp();
+  }
+
+  // ------------------------------------------------ softmax and top-K ------
+  const bool got = __all_sync(0xffffffffu, wait_bounded(done_bar, 0, abort_p, status) ? 1 : 0);
+  tc_fence_after();
+  const int r = warp * 32 + lane;
+  const int64_t t = static_cast<int64_t>(m0) + r;
+  const bool live = t < T;
+  const uint32_t trow = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+  const int nch = (np + 31) / 32;
+  const bool select_only = (flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
+
+  if (!got) {
+    // results stay in range for the stages downstream; the status word says
+    // that they are not to be used
+    if (live)
+      for (int k = 0; k < K; ++k) {
+        idx[t * K + k] = k;
+        w[t * K + k] = 0.0f;
+      }
+  } else if (NCH == 0) {
+    float m = -CUDART_INF_F;
+#pragma unroll 1
+    for (int c = 0; c < nch; ++c) {
+      float x[32];
+      tmem_ld32(trow + c * 32, x);
+      tmem_ld_wait_regs(x);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int e = c * 32 + j;
+        if (e < n) m = fmaxf(m, select_only ? x[j] : x[j] + sbias[e]);
+      }
+    }
+    float z = 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < nch; ++c) {
+      float x[32];
+      tmem_ld32(trow + c * 32, x);
+      tmem_ld_wait_regs(x);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int e = c * 32 + j;
+        if (e < n) z += expf((select_only ? x[j] : x[j] + sbias[e]) - m);
+      }
+    }
+    const float inv_z = 1.0f / z;
+
+    float pv = CUDART_INF_F;  // previous pick (key, index)
+    int pe = -1;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+      float bv = -CUDART_INF_F, blg = 0.0f;
+      int bi = -1;
+#pragma unroll 1
+      for (int c = 0; c < nch; ++c) {
+        float x[32];
+        tmem_ld32(trow + c * 32, x);
+        tmem_ld_wait_regs(x);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int e = c * 32 + j;
+          const float key = x[j] + sbias[e];
+          const bool after = key < pv || (key == pv && e > pe);
+          if (e < n && after && (bi < 0 || key > bv)) {
+            bv = key;
+            bi = e;
+            blg = select_only ? x[j] : key;
+          }
+        }
+      }
+      if (live) {
+        idx[t * K + k] = bi;
+        w[t * K + k] = expf(blg - m) * inv_z;
+      }
+      pv = bv;
+      pe = bi;
+    }
+
+    if (STATS) {
+      // scores of this warp's 32 tokens, transposed through shared memory
+      // (the ring is free: every MMA that read it has completed)
+      const int ld = np + 1;
+      float* sc = reinterpret_cast<float*>(smem) + warp * 32 * ld;
+#pragma unroll 1
+      for (int c = 0; c < nch; ++c) {
+        float x[32];
+        tmem_ld32(trow + c * 32, x);
+        tmem_ld_wait_regs(x);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int e = c * 32 + j;
+          if (e < np)
+            sc[lane * ld + e] =
+                (live && e < n) ? expf((select_only ? x[j] : x[j] + sbias[e]) - m) / z : 0.0f;
+        }
+      }
+      __syncwarp();
+      const int64_t g = static_cast<int64_t>(blockIdx.x) * (kRtTokens / 32) + warp;
+      if (g * 32 < T) {
+        for (int e = lane; e < n; e += 32) {
+          float a = 0.0f;
+          for (int tok = 0; tok < 32; ++tok) a += sc[tok * ld + e];
+          pstat[g * n + e] = a;
+        }
+      }
+    }
+  } else {
+    // logits -> selection keys (and, with SEL, the softmax logits) in registers
+    constexpr int NR = (NCH > 0 ? NCH : 1) * 32;
+    float key[NR];
+    float lg[SEL ? NR : 1];
+#pragma unroll
+    for (int c = 0; c < NR / 32; ++c) tmem_ld32(trow + c * 32, key + c * 32);
+#pragma unroll
+    for (int c = 0; c < NR / 32; ++c) tmem_ld_wait_regs(key + c * 32);
+    float m = -CUDART_INF_F;
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+      if (SEL) lg[j] = j < n ? key[j] : -CUDART_INF_F;
+      key[j] = j < n ? key[j] + sbias[j] : -CUDART_INF_F;
+      m = fmaxf(m, SEL ? lg[j] : key[j]);
+    }
+    float z = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NR; ++j) z += expf((SEL ? lg[j] : key[j]) - m);
+    const float inv_z = 1.0f / z;
+
+    float pv = CUDART_INF_F;  // previous pick (key, index)
+    int pe = -1;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+      float bv = -CUDART_INF_F, blg = 0.0f;
+      int bi = -1;
+#pragma unroll
+      for (int j = 0; j < NR; ++j) {
+        const float kj = key[j];
+        const bool after = kj < pv || (kj == pv && j > pe);
+        if (after && kj > bv) {
+          bv = kj;
+          bi = j;
+          blg = SEL ? lg[j] : kj;
+        }
+      }
+      if (live) {
+        idx[t * K + k] = bi;
+        w[t * K + k] = expf(blg - m) * inv_z;
+      }
+      pv = bv;
+      pe = bi;
+    }
+
+    if (STATS) {
+      const int ld = np + 1;
+      float* sc = reinterpret_cast<float*>(smem) + warp * 32 * ld;
+#pragma unroll
+      for (int j = 0; j < NR; ++j)
+        if (j < np) sc[lane * ld + j] = (live && j < n) ? expf((SEL ? lg[j] : key[j]) - m) / z : 0.0f;
+      __syncwarp();
+      const int64_t g = static_cast<int64_t>(blockIdx.x) * (kRtTokens / 32) + warp;
+      if (g * 32 < T) {
+        for (int e = lane; e < n; e += 32) {
+          float a = 0.0f;
+          for (int tok = 0; tok < 32; ++tok) a += sc[tok * ld + e];
+          pstat[g * n + e] = a;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+}  // namespace
+
+int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T, int d, int n,
+                     int K, int flags, int32_t* idx, float* w, float* pstat, int32_t* status,
+                     cudaStream_t st) {
+  if (T == 0) return MOE_OK;
+  if (d % kRtBK != 0 || n < 1 || n > 256) return MOE_ERR_SHAPE;
+  const int np = rt_padded_experts(n);
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(np)) cols *= 2;
+  const int stages = rt_stages(np);
+  const int smem = stages * rt_stage_bytes(np) + 1024;
+  CUtensorMap mu, me;
+  if (!make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u, static_cast<uint64_t>(d),
+                   static_cast<uint64_t>(T), static_cast<uint64_t>(d) * 2, kRtBK, kRtTokens) ||
+      !make_map_2d(&me, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, E, static_cast<uint64_t>(d),
+                   static_cast<uint64_t>(n), static_cast<uint64_t>(d) * 2, kRtBK,
+                   static_cast<uint32_t>(np)))
+    return MOE_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>((T + kRtTokens - 1) / kRtTokens);
+  auto go = [&](auto kern, bool& attr_done) -> int {
+    // one opt-in size covering every expert count (smem never exceeds it)
+    if (!attr_done) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kRtSmemBudget + 1024) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      attr_done = true;
+    }
+    kern<<<grid, kRtThreads, smem, st>>>(mu, me, bias, T, d, n, np, K, flags, stages, cols, idx,
+                                         w, pstat, status);
+    count_launch();
+    return check_launch();
+  };
+  const bool sel = (flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
+  const int nch = (np + 31) / 32;
+  // register-resident variants up to 64 experts (128 without SEL)
+  // (with statistics, beyond 64 experts the register variant would spill)
+  const int v = (nch <= 2 || (nch <= 4 && !sel && !pstat)) ? nch : 0;
+#define MOE_RT_GO(STATS, NCH, SEL)                                  \
+  {                                                                 \
+    static bool done = false;                                       \
+    return go(router_tc_kernel<STATS, NCH, SEL>, done);             \
+  }
+#define MOE_RT_VARIANTS(STATS)                                      \
+  if (v == 1 && sel) MOE_RT_GO(STATS, 1, true)                      \
+  if (v == 1) MOE_RT_GO(STATS, 1, false)                            \
+  if (v == 2 && sel) MOE_RT_GO(STATS, 2, true)                      \
+  if (v == 2) MOE_RT_GO(STATS, 2, false)                            \
+  if (v == 3) MOE_RT_GO(STATS, (STATS ? 0 : 3), false)              \
+  if (v == 4) MOE_RT_GO(STATS, (STATS ? 0 : 4), false)              \
+  MOE_RT_GO(STATS, 0, false)
+  if (pstat) {
+    MOE_RT_VARIANTS(true)
+  } else {
+    MOE_RT_VARIANTS(false)
+  }
+#undef MOE_RT_VARIANTS
+#undef MOE_RT_GO
+}
+
+}  // namespace moe

@@ -155,3 +155,78 @@ def test_expert_balance_statistics():
     np.testing.assert_allclose(to_numpy(f), f_ref, rtol=1e-6)
     np.testing.assert_allclose(to_numpy(Pm), P_ref, rtol=1e-4, atol=1e-7)
     np.testing.assert_allclose(to_numpy(f).sum(), 24.0, rtol=1e-5)
+
+
+@pytest.mark.parametrize("wl", CASES[:3], ids=[c.name for c in CASES[:3]])
+def test_simt_router_full(wl):
+    """The CUDA-core router (MOE_FLAG_ROUTER_SIMT) meets the same bars."""
+    P.full_parity(S.make_inputs(wl), flags=L.MOE_FLAG_ROUTER_SIMT)
+
+
+# expert counts that reach every epilogue variant of the tensor-core router:
+# 1, 2, 3 and 4 register chunks, and the chunked path (256 experts, or
+# select-only bias beyond 64 experts)
+ROUTER_CASES = CASES + [
+    W("router_90", T=300, d=256, n_routed=90, n_shared=1, inter=64, top_k=6, bias_var=0.5),
+    W("router_128", T=300, d=256, n_routed=128, n_shared=1, inter=64, top_k=12),
+    W("router_256", T=300, d=256, n_routed=256, n_shared=1, inter=64, top_k=8),
+]
+ROUTER_FLAGS = {"bias_in_softmax": 0, "bias_select_only": L.MOE_FLAG_BIAS_SELECT_ONLY}
+
+
+@pytest.mark.parametrize("bias_mode", sorted(ROUTER_FLAGS))
+@pytest.mark.parametrize("wl", ROUTER_CASES, ids=[c.name for c in ROUTER_CASES])
+def test_tensor_core_and_simt_routers_agree(wl, bias_mode):
+    """Both routers compute the same logits up to fp32 summation order: the
+    same experts for every token without a near tie in the oracle's scores,
+    gates within the fp32 gate bar."""
+    from oracle import moe_oracle as O
+    if bias_mode == "bias_select_only" and wl.bias_var == 0:
+        wl = S.custom_workload(wl.name + "_b", T=wl.T, d=wl.d, n_routed=wl.n_routed,
+                               n_shared=wl.n_shared, inter=wl.inter, top_k=wl.top_k, bias_var=0.5)
+    x = S.make_inputs(wl)
+    layer = MoELayer(x, "cuda:0")
+    u = to_device(x.u, "cuda:0")
+    bf = ROUTER_FLAGS[bias_mode]
+    out = {}
+    for name, fl in (("tc", bf), ("simt", bf | L.MOE_FLAG_ROUTER_SIMT)):
+        sh = L.make_shape(wl.T, wl.d, wl.n_routed, wl.n_shared, wl.inter, wl.top_k, flags=fl)
+        idx = torch.full((wl.T, wl.top_k), -1, dtype=torch.int32, device="cuda:0")
+        w = torch.full((wl.T, wl.top_k), -1.0, dtype=torch.float32, device="cuda:0")
+        L.moe_route(sh, u, layer.E, layer.bias, idx, w)
+        torch.cuda.synchronize()
+        out[name] = (to_numpy(idx), to_numpy(w))
+    fx = P.f64_inputs(x)
+    s = O.softmax(O.router_logits(fx["u"], fx["E"], fx["bias"]))
+    near = P.near_tie_tokens(s, wl.top_k)
+    if bias_mode == "bias_select_only":
+        ref_idx, _ = O.topk_gates_select_only_bias(O.router_logits(fx["u"], fx["E"], None),
+                                                   fx["bias"], wl.top_k)
+        assert np.all((out["tc"][0] == ref_idx).all(axis=1) | near)
+    same = np.all(out["tc"][0] == out["simt"][0], axis=1)
+    assert np.all(same | near)
+    ok = same & ~near
+    np.testing.assert_allclose(out["tc"][1][ok], out["simt"][1][ok], rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("n", [24, 90, 200])
+def test_balance_statistics_every_router_variant(n):
+    """Eqs. (12)-(13) through the statistics variants of the router
+    (register-resident up to 64 experts, chunked beyond)."""
+    from oracle import moe_oracle as O
+    wl = W(f"bal{n}", T=700, d=256, n_routed=n, n_shared=1, inter=64, top_k=4, bias_var=0.3)
+    x = S.make_inputs(wl)
+    rep = P.full_parity(x)
+    layer = rep["gpu"]["layer"]
+    dev = layer.device
+    counts = to_device(rep["gpu"]["counts"], dev)
+    f = torch.empty(n, dtype=torch.float32, device=dev)
+    Pm = torch.empty(n, dtype=torch.float32, device=dev)
+    L.moe_expert_balance(layer.shape, to_device(x.u, dev), layer.E, layer.bias, counts, f, Pm,
+                         layer.ws)
+    torch.cuda.synchronize()
+    fx = P.f64_inputs(x)
+    s = O.softmax(O.router_logits(fx["u"], fx["E"], fx["bias"]))
+    f_ref, P_ref, _ = O.expert_balance(s, rep["gpu"]["idx"])
+    np.testing.assert_allclose(to_numpy(f), f_ref, rtol=1e-6)
+    np.testing.assert_allclose(to_numpy(Pm), P_ref, rtol=1e-4, atol=1e-7)
