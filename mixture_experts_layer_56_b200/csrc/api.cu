@@ -223,6 +223,8 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
   if (s.flags & MOE_FLAG_GEMM_SINGLE_CTA) pair = false;
   if (s.flags & MOE_FLAG_GEMM_CTA_PAIR) pair = true;
   const int BM = pair ? 256 : 128;
+  // rows of an A box: below 128 tokens no group has more than T rows
+  const uint32_t a_rows = pair || T >= 128 ? 128u : static_cast<uint32_t>((T + 7) / 8 * 8);
   const int64_t routed_mt_ub = (rows + BM - 1) / BM + (rows < n ? rows : n);
   const int64_t shared_mt = ns > 0 ? (T + BM - 1) / BM : 0;
   auto launch = [&](int BN, int epi, const GemmMaps& m, const GroupedGemmArgs& a) {
@@ -250,10 +252,10 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     const int BN = pick_bn(2 * I, 2 * I * ns, (2 * I) % 256 == 0 ? 256 : 128, 128);
     const uint32_t bbox = pair ? BN / 2 : BN;
     GemmMaps m;
-    bool ok = make_map_bf16(&m.a_r, 2, xperm, d64, rows, 1, d64 * 2, 0, 128) &&
+    bool ok = make_map_bf16(&m.a_r, 2, xperm, d64, rows, 1, d64 * 2, 0, a_rows) &&
               make_map_bf16(&m.b_r, 3, W13, d64, 2 * I64, n, d64 * 2, 2 * I64 * d64 * 2, bbox);
     if (ns > 0) {
-      ok = ok && make_map_bf16(&m.a_s, 2, u, d64, T, 1, d64 * 2, 0, 128) &&
+      ok = ok && make_map_bf16(&m.a_s, 2, u, d64, T, 1, d64 * 2, 0, a_rows) &&
            make_map_bf16(&m.b_s, 3, W13_s, d64, 2 * I64 * ns, 1, d64 * 2, 2 * I64 * ns * d64 * 2,
                          bbox);
     } else {
@@ -275,6 +277,7 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     a.out_s = act_s;
     a.ld_s = static_cast<int64_t>(I) * ns;
     a.status = status;
+    a.a_rows = static_cast<int32_t>(a_rows);
     Stage sg(MOE_KERNEL_GEMM_GATE_UP, st);
     if (int rc = launch(BN, kEpiSwiGLU, m, a)) return rc;
   }
@@ -283,10 +286,10 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     const int BN = pick_bn(d, d, d % 256 == 0 ? 256 : (d % 128 == 0 ? 128 : 64), 64);
     const uint32_t bbox = pair ? BN / 2 : BN;
     GemmMaps m;
-    bool ok = make_map_bf16(&m.a_r, 2, act, I64, rows, 1, I64 * 2, 0, 128) &&
+    bool ok = make_map_bf16(&m.a_r, 2, act, I64, rows, 1, I64 * 2, 0, a_rows) &&
               make_map_bf16(&m.b_r, 3, W2, I64, d64, n, I64 * 2, d64 * I64 * 2, bbox);
     if (ns > 0) {
-      ok = ok && make_map_bf16(&m.a_s, 2, act_s, I64 * ns, T, 1, I64 * ns * 2, 0, 128) &&
+      ok = ok && make_map_bf16(&m.a_s, 2, act_s, I64 * ns, T, 1, I64 * ns * 2, 0, a_rows) &&
            make_map_bf16(&m.b_s, 3, W2_s, I64, d64, ns, I64 * 2, d64 * I64 * 2, bbox);
     } else {
       m.a_s = m.a_r;
@@ -308,6 +311,7 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     a.out_s = ysh;
     a.ld_s = d;
     a.status = status;
+    a.a_rows = static_cast<int32_t>(a_rows);
     Stage sg(MOE_KERNEL_GEMM_DOWN, st);
     if (int rc = launch(BN, kEpiPlain, m, a)) return rc;
   }

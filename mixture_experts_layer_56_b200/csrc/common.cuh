@@ -72,10 +72,55 @@ __device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
   if (status) *reinterpret_cast<volatile int32_t*>(status) = code;
 }
 
+// Programmatic dependent launch.  A kernel started by launch_k() may begin
+// while the kernel before it in the stream is still running.  pdl_wait()
+// blocks until that kernel has completed and its writes are visible, so it
+// must precede the first read or write of global memory that earlier
+// stream work may touch; only set-up (barriers, TMEM, descriptor prefetch)
+// goes before it.  pdl_trigger() lets the next kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // host-side bookkeeping shared by the launch wrappers
 // ---------------------------------------------------------------------------
 void count_launch(int n = 1);
 int check_launch();  // MOE_OK or MOE_ERR_CUDA after a <<<>>> launch
+
+// Launch with programmatic stream serialisation (the kernel must call
+// pdl_wait() before touching global memory) and, if cluster > 1, thread
+// block clusters of that many CTAs along x.
+template <typename... KArgs, typename... Args>
+int launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+             unsigned cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (cluster > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = cluster;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  count_launch();
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return check_launch();
+}
 
 }  // namespace moe

@@ -129,6 +129,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     tmem_alloc(smem_addr(&tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_wait();  // offsets, operands and outputs belong to earlier stream work
+  pdl_trigger();
   for (int g = tid; g < G; g += kThreads) {
     int rows, row0, nt;
     if (hs && g == 0) {
@@ -178,6 +180,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
         tma_prefetch_desc(&tmA_s);
         tma_prefetch_desc(&tmB_s);
       }
+      const uint32_t a_bytes =
+          static_cast<uint32_t>(args.a_rows > 0 && args.a_rows < BM ? args.a_rows : BM) * BK * 2;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, issued_parity = 0;
@@ -193,7 +197,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
         for (int kb = 0; kb < nkb; ++kb) {
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_p, args.status)) { ok = false; break; }
           const uint32_t sa = smem_base + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
+          mbar_arrive_expect_tx(full_bar(stage), a_bytes + B_BYTES);
           tma_load_2d(sa, ma, full_bar(stage), kb * BK, row);
           tma_load_3d(sa + A_BYTES, mb, full_bar(stage), (kb % args.kb_per_expert) * BK, nrow,
                       zbase + kb / args.kb_per_expert);
@@ -395,9 +399,8 @@ static int launch_impl(const GemmMaps& m, const GroupedGemmArgs& args, int grid,
       return MOE_ERR_CUDA;
     attr_done = true;
   }
-  kern<<<grid, kThreads, smem_bytes<BN>(), stream>>>(m.a_r, m.a_s, m.b_r, m.b_s, args);
-  count_launch();
-  return check_launch();
+  return launch_k(kern, grid, kThreads, smem_bytes<BN>(), stream, 1, m.a_r, m.a_s, m.b_r, m.b_s,
+                  args);
 }
 
 int launch_grouped_gemm(int BN, int epi, const GemmMaps& maps, const GroupedGemmArgs& args,

@@ -27,6 +27,11 @@ struct GroupedGemmArgs {
   void* out_s;             // shared output: bf16 (SwiGLU) or fp32 (plain)
   int64_t ld_s;
   int32_t* status;         // workspace status word
+  // Rows in the A maps' box (single-CTA kernel; 0 means 128).  Smaller for
+  // batches of fewer than 128 tokens, where no group has more rows: the
+  // tile's other A rows are left as they are in shared memory and their
+  // accumulator rows are never stored.
+  int32_t a_rows;
 };
 
 // A maps: rank 2 {K, rows}; B maps: rank 3 {K, N rows, experts}; bf16, box

@@ -165,6 +165,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
     tmem_alloc_pair(smem_addr(&tmem_slot), TMEM_COLS);
     tmem_relinquish_pair();
   }
+  pdl_wait();  // offsets, operands and outputs belong to earlier stream work
+  pdl_trigger();
   for (int g = tid; g < G; g += kPairThreads) {
     int rows, row0, nt;
     if (hs && g == 0) {
@@ -425,22 +427,8 @@ int launch_pair_impl(const GemmMaps& m, const GroupedGemmArgs& args, int cluster
       return MOE_ERR_CUDA;
     attr_done = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * clusters, 1, 1);
-  cfg.blockDim = dim3(kPairThreads, 1, 1);
-  cfg.dynamicSmemBytes = pair_smem_bytes<BN, EPI>();
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, m.a_r, m.a_s, m.b_r, m.b_s, args) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  count_launch();
-  return check_launch();
+  return launch_k(kern, dim3(2 * clusters), kPairThreads, pair_smem_bytes<BN, EPI>(), stream, 2,
+                  m.a_r, m.a_s, m.b_r, m.b_s, args);
 }
 
 }  // namespace

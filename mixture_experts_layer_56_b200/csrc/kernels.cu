@@ -56,6 +56,8 @@ __global__ void __launch_bounds__(kDispThreads)
 dispatch_count_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n,
                       int32_t* __restrict__ chunk_counts) {
   __shared__ int wc[kDispWarps][256];
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispThreads + threadIdx.x;
   uint32_t mask[NW];
@@ -75,6 +77,8 @@ dispatch_scan_kernel(const int32_t* __restrict__ chunk_counts, int64_t nchunks, 
                      int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
                      int32_t* __restrict__ offsets) {
   __shared__ int tot[256];
+  pdl_wait();
+  pdl_trigger();
   __shared__ int off[257];
   const int e = threadIdx.x;
   // pass 1: tokens per expert (loads batched so that 8 are in flight)
@@ -135,6 +139,8 @@ dispatch_scatter_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n
                         const int32_t* __restrict__ chunk_base, int32_t* __restrict__ perm,
                         int32_t* __restrict__ inv) {
   __shared__ int wc[kDispWarps][256];
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispThreads + threadIdx.x;
   // this token's experts, kept in registers
@@ -190,6 +196,8 @@ dispatch_single_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n,
                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                        int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
   __shared__ int wc[kDispWarps][256];
+  pdl_wait();
+  pdl_trigger();
   __shared__ int tot[256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = threadIdx.x;
@@ -265,6 +273,8 @@ __global__ void __launch_bounds__(256)
 gather_rows_kernel(const T* __restrict__ u, const int32_t* __restrict__ perm, int64_t rows, int d,
                    int K, T* __restrict__ xperm) {
   constexpr int V = Vec16<T>::N;
+  pdl_wait();
+  pdl_trigger();
   constexpr int U = 4;  // 16-byte loads in flight per lane before the stores
   const int lane = threadIdx.x & 31;
   const int nv = d / V;
@@ -301,6 +311,8 @@ combine_kernel(const T* __restrict__ u, const float* __restrict__ ysh, const T* 
                const float* __restrict__ w, const int32_t* __restrict__ inv, int64_t Tn, int d,
                int K, T* __restrict__ h) {
   // one warp per (token, block of 32*V columns)
+  pdl_wait();
+  pdl_trigger();
   constexpr int V = Vec16<T>::N;
   const int lane = threadIdx.x & 31;
   const int nblk = (d + 32 * V - 1) / (32 * V);
@@ -531,29 +543,25 @@ int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_
     // one block does it all
 #define MOE_SINGLE_CASE(W)                                                                   \
   case W:                                                                                    \
-    if (K <= 8)                                                                              \
-      dispatch_single_kernel<W, 8><<<1, kDispThreads, 0, st>>>(idx, T, K, n, counts, offsets,  \
-                                                               perm, inv);                   \
-    else if (K <= 16)                                                                        \
-      dispatch_single_kernel<W, 16><<<1, kDispThreads, 0, st>>>(idx, T, K, n, counts, offsets, \
-                                                                perm, inv);                  \
-    else                                                                                     \
-      dispatch_single_kernel<W, 32><<<1, kDispThreads, 0, st>>>(idx, T, K, n, counts, offsets, \
-                                                                perm, inv);                  \
-    break;
+    return K <= 8    ? launch_k(dispatch_single_kernel<W, 8>, 1, kDispThreads, 0, st, 1, idx, T, K, \
+                                n, counts, offsets, perm, inv)                               \
+           : K <= 16 ? launch_k(dispatch_single_kernel<W, 16>, 1, kDispThreads, 0, st, 1, idx, T,  \
+                                K, n, counts, offsets, perm, inv)                            \
+                     : launch_k(dispatch_single_kernel<W, 32>, 1, kDispThreads, 0, st, 1, idx, T,  \
+                                K, n, counts, offsets, perm, inv);
     switch (nw) {
       MOE_SINGLE_CASE(1) MOE_SINGLE_CASE(2) MOE_SINGLE_CASE(3) MOE_SINGLE_CASE(4)
       MOE_SINGLE_CASE(5) MOE_SINGLE_CASE(6) MOE_SINGLE_CASE(7) MOE_SINGLE_CASE(8)
       default: return MOE_ERR_SHAPE;
     }
 #undef MOE_SINGLE_CASE
-    count_launch();
-    return check_launch();
   }
+  const dim3 grid(static_cast<unsigned>(nch));
+  int rc = MOE_ERR_SHAPE;
 #define MOE_DISPATCH_CASE(W)                                                                 \
   case W:                                                                                    \
-    dispatch_count_kernel<W><<<static_cast<unsigned>(nch), kDispThreads, 0, st>>>(idx, T, K, n, \
-                                                                                  chunk_counts); \
+    rc = launch_k(dispatch_count_kernel<W>, grid, kDispThreads, 0, st, 1, idx, T, K, n,      \
+                  chunk_counts);                                                             \
     break;
   switch (nw) {
     MOE_DISPATCH_CASE(1) MOE_DISPATCH_CASE(2) MOE_DISPATCH_CASE(3) MOE_DISPATCH_CASE(4)
@@ -561,22 +569,19 @@ int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_
     default: return MOE_ERR_SHAPE;
   }
 #undef MOE_DISPATCH_CASE
-  count_launch();
-  if (int rc = check_launch()) return rc;
-  dispatch_scan_kernel<<<1, 256, 0, st>>>(chunk_counts, nch, n, chunk_base, counts, offsets);
-  count_launch();
-  if (int rc = check_launch()) return rc;
+  if (rc) return rc;
+  if (int r2 = launch_k(dispatch_scan_kernel, 1, 256, 0, st, 1, static_cast<const int32_t*>(chunk_counts),
+                        nch, n, chunk_base, counts, offsets))
+    return r2;
+  rc = MOE_ERR_SHAPE;
 #define MOE_SCATTER_CASE(W)                                                                  \
   case W:                                                                                    \
-    if (K <= 8)                                                                              \
-      dispatch_scatter_kernel<W, 8><<<static_cast<unsigned>(nch), kDispThreads, 0, st>>>(     \
-          idx, T, K, n, chunk_base, perm, inv);                                              \
-    else if (K <= 16)                                                                        \
-      dispatch_scatter_kernel<W, 16><<<static_cast<unsigned>(nch), kDispThreads, 0, st>>>(    \
-          idx, T, K, n, chunk_base, perm, inv);                                              \
-    else                                                                                     \
-      dispatch_scatter_kernel<W, 32><<<static_cast<unsigned>(nch), kDispThreads, 0, st>>>(    \
-          idx, T, K, n, chunk_base, perm, inv);                                              \
+    rc = K <= 8    ? launch_k(dispatch_scatter_kernel<W, 8>, grid, kDispThreads, 0, st, 1, idx, T, \
+                              K, n, static_cast<const int32_t*>(chunk_base), perm, inv)      \
+         : K <= 16 ? launch_k(dispatch_scatter_kernel<W, 16>, grid, kDispThreads, 0, st, 1, idx,   \
+                              T, K, n, static_cast<const int32_t*>(chunk_base), perm, inv)   \
+                   : launch_k(dispatch_scatter_kernel<W, 32>, grid, kDispThreads, 0, st, 1, idx,   \
+                              T, K, n, static_cast<const int32_t*>(chunk_base), perm, inv);  \
     break;
   switch (nw) {
     MOE_SCATTER_CASE(1) MOE_SCATTER_CASE(2) MOE_SCATTER_CASE(3) MOE_SCATTER_CASE(4)
@@ -584,8 +589,7 @@ int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_
     default: return MOE_ERR_SHAPE;
   }
 #undef MOE_SCATTER_CASE
-  count_launch();
-  return check_launch();
+  return rc;
 }
 
 int launch_gather(int dtype, const void* u, const int32_t* perm, int64_t rows, int d, int K,
@@ -593,13 +597,10 @@ int launch_gather(int dtype, const void* u, const int32_t* perm, int64_t rows, i
   if (rows == 0) return MOE_OK;
   const unsigned grid = grid_for_rows(rows, 8);
   if (dtype == MOE_DTYPE_BF16)
-    gather_rows_kernel<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16*>(u), perm, rows, d, K,
-                                                   static_cast<bf16*>(xperm));
-  else
-    gather_rows_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(u), perm, rows, d, K,
-                                                    static_cast<float*>(xperm));
-  count_launch();
-  return check_launch();
+    return launch_k(gather_rows_kernel<bf16>, grid, 256, 0, st, 1, static_cast<const bf16*>(u),
+                    perm, rows, d, K, static_cast<bf16*>(xperm));
+  return launch_k(gather_rows_kernel<float>, grid, 256, 0, st, 1, static_cast<const float*>(u),
+                  perm, rows, d, K, static_cast<float*>(xperm));
 }
 
 int launch_combine(int dtype, const void* u, const float* ysh, const void* y, const float* w,
@@ -608,15 +609,10 @@ int launch_combine(int dtype, const void* u, const float* ysh, const void* y, co
   const int V = dtype == MOE_DTYPE_BF16 ? 8 : 4;
   const unsigned grid = grid_for_rows(T * ((d + 32 * V - 1) / (32 * V)), 8);
   if (dtype == MOE_DTYPE_BF16)
-    combine_kernel<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16*>(u), ysh,
-                                               static_cast<const bf16*>(y), w, inv, T, d, K,
-                                               static_cast<bf16*>(h));
-  else
-    combine_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(u), ysh,
-                                                static_cast<const float*>(y), w, inv, T, d, K,
-                                                static_cast<float*>(h));
-  count_launch();
-  return check_launch();
+    return launch_k(combine_kernel<bf16>, grid, 256, 0, st, 1, static_cast<const bf16*>(u), ysh,
+                    static_cast<const bf16*>(y), w, inv, T, d, K, static_cast<bf16*>(h));
+  return launch_k(combine_kernel<float>, grid, 256, 0, st, 1, static_cast<const float*>(u), ysh,
+                  static_cast<const float*>(y), w, inv, T, d, K, static_cast<float*>(h));
 }
 
 int launch_pack_w13(int dtype, const void* W1, const void* W3, void* W13, int n_experts, int I,

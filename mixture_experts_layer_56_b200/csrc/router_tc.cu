@@ -88,11 +88,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
     fence_mbar_init();
     fence_async_shared();
   }
-  for (int e = tid; e < 256; e += kRtThreads) sbias[e] = (bias != nullptr && e < n) ? bias[e] : 0.0f;
   if (warp == 2) {
     tmem_alloc(smem_addr(&tmem_slot), tmem_cols);
     tmem_relinquish();
   }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmU);
+    tma_prefetch_desc(&tmE);
+  }
+  pdl_wait();  // u, E, bias and the outputs belong to earlier stream work
+  for (int e = tid; e < 256; e += kRtThreads) sbias[e] = (bias != nullptr && e < n) ? bias[e] : 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -102,8 +107,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer ----
     if (lane == 0) {
-      tma_prefetch_desc(&tmU);
-      tma_prefetch_desc(&tmE);
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_parity = 0;
       bool ok = true;
@@ -158,6 +161,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
   }
 
   // ------------------------------------------------ softmax and top-K ------
+  pdl_trigger();
   const bool got = __all_sync(0xffffffffu, wait_bounded(done_bar, 0, abort_p, status) ? 1 : 0);
   tc_fence_after();
   const int r = warp * 32 + lane;
@@ -270,41 +274,25 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
     for (int c = 0; c < NR / 32; ++c) tmem_ld32(trow + c * 32, key + c * 32);
 #pragma unroll
     for (int c = 0; c < NR / 32; ++c) tmem_ld_wait_regs(key + c * 32);
-    float m = -CUDART_INF_F;
+    // four interleaved chains (j mod 4) keep the scans short in latency
+    constexpr int NB = 4;
+    float mb[NB];
+#pragma unroll
+    for (int q = 0; q < NB; ++q) mb[q] = -CUDART_INF_F;
 #pragma unroll
     for (int j = 0; j < NR; ++j) {
       if (SEL) lg[j] = j < n ? key[j] : -CUDART_INF_F;
       key[j] = j < n ? key[j] + sbias[j] : -CUDART_INF_F;
-      m = fmaxf(m, SEL ? lg[j] : key[j]);
+      mb[j % NB] = fmaxf(mb[j % NB], SEL ? lg[j] : key[j]);
     }
-    float z = 0.0f;
+    const float m = fmaxf(fmaxf(mb[0], mb[1]), fmaxf(mb[2], mb[3]));
+    float zb[NB];
 #pragma unroll
-    for (int j = 0; j < NR; ++j) z += expf((SEL ? lg[j] : key[j]) - m);
+    for (int q = 0; q < NB; ++q) zb[q] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NR; ++j) zb[j % NB] += expf((SEL ? lg[j] : key[j]) - m);
+    const float z = (zb[0] + zb[1]) + (zb[2] + zb[3]);
     const float inv_z = 1.0f / z;
-
-    float pv = CUDART_INF_F;  // previous pick (key, index)
-    int pe = -1;
-#pragma unroll 1
-    for (int k = 0; k < K; ++k) {
-      float bv = -CUDART_INF_F, blg = 0.0f;
-      int bi = -1;
-#pragma unroll
-      for (int j = 0; j < NR; ++j) {
-        const float kj = key[j];
-        const bool after = kj < pv || (kj == pv && j > pe);
-        if (after && kj > bv) {
-          bv = kj;
-          bi = j;
-          blg = SEL ? lg[j] : kj;
-        }
-      }
-      if (live) {
-        idx[t * K + k] = bi;
-        w[t * K + k] = expf(blg - m) * inv_z;
-      }
-      pv = bv;
-      pe = bi;
-    }
 
     if (STATS) {
       const int ld = np + 1;
@@ -321,6 +309,48 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
           pstat[g * n + e] = a;
         }
       }
+    }
+
+    // K passes; each takes the largest remaining key (lower index first on
+    // equal keys) and removes it from the next pass
+    int prev = -1;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+      float bv[NB], bl[NB];
+      int bi[NB];
+#pragma unroll
+      for (int q = 0; q < NB; ++q) {
+        bv[q] = -CUDART_INF_F;
+        bl[q] = 0.0f;
+        bi[q] = 0x7fffffff;
+      }
+#pragma unroll
+      for (int j = 0; j < NR; ++j) {
+        const int q = j % NB;
+        const float kj = (j == prev) ? -CUDART_INF_F : key[j];
+        key[j] = kj;
+        if (kj > bv[q]) {
+          bv[q] = kj;
+          bi[q] = j;
+          if (SEL) bl[q] = lg[j];
+        }
+      }
+      // merge the chains: larger key, then lower index
+      float v = bv[0], l = bl[0];
+      int e = bi[0];
+#pragma unroll
+      for (int q = 1; q < NB; ++q) {
+        if (bv[q] > v || (bv[q] == v && bi[q] < e)) {
+          v = bv[q];
+          e = bi[q];
+          l = bl[q];
+        }
+      }
+      if (live) {
+        idx[t * K + k] = e;
+        w[t * K + k] = expf((SEL ? l : v) - m) * inv_z;
+      }
+      prev = e;
     }
   }
 
@@ -360,10 +390,8 @@ int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T,
         return MOE_ERR_CUDA;
       attr_done = true;
     }
-    kern<<<grid, kRtThreads, smem, st>>>(mu, me, bias, T, d, n, np, K, flags, stages, cols, idx,
-                                         w, pstat, status);
-    count_launch();
-    return check_launch();
+    return launch_k(kern, grid, kRtThreads, static_cast<size_t>(smem), st, 1, mu, me, bias, T, d,
+                    n, np, K, flags, stages, cols, idx, w, pstat, status);
   };
   const bool sel = (flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
   const int nch = (np + 31) / 32;
