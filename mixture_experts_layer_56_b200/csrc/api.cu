@@ -331,16 +331,20 @@ int forward_device(const moe_shape_t& s, const Layout& L, const void* u, const v
   int32_t* inv = at<int32_t>(ws, L.inv);
   void* y = at<void>(ws, L.y);
   float* ysh = at<float>(ws, L.ysh);
+  // batches of more than one dispatch chunk: the router also counts
+  int32_t* chunk_counts = at<int32_t>(ws, L.chunk_counts);
+  bool counted = false;
   {
     Stage sg(MOE_KERNEL_ROUTER, st);
     if (int rc = launch_router(s.dtype, u, E, bias, T, s.d, n, K, s.flags, idx, w, nullptr,
-                               at<int32_t>(ws, L.status), st))
+                               at<int32_t>(ws, L.status), st,
+                               T > kDispatchChunk ? chunk_counts : nullptr, &counted))
       return rc;
   }
   {
     Stage sg(MOE_KERNEL_DISPATCH, st);
-    if (int rc = launch_dispatch(idx, T, K, n, at<int32_t>(ws, L.chunk_counts),
-                                 at<int32_t>(ws, L.chunk_base), counts, offsets, perm, inv, st))
+    if (int rc = launch_dispatch(idx, T, K, n, chunk_counts, at<int32_t>(ws, L.chunk_base), counts,
+                                 offsets, perm, inv, st, counted))
       return rc;
   }
   // the tensor-core path writes y in token-slot order (the combine then

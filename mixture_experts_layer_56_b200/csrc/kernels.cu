@@ -529,7 +529,7 @@ inline unsigned grid_for_rows(int64_t rows, int rows_per_block) {
 
 int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_counts,
                     int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* perm,
-                    int32_t* inv, cudaStream_t st) {
+                    int32_t* inv, cudaStream_t st, bool counts_ready) {
   const int64_t nch = dispatch_num_chunks(T);
   const int nw = (n + 31) / 32;
   if (T == 0) {
@@ -563,10 +563,14 @@ int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_
     rc = launch_k(dispatch_count_kernel<W>, grid, kDispThreads, 0, st, 1, idx, T, K, n,      \
                   chunk_counts);                                                             \
     break;
-  switch (nw) {
-    MOE_DISPATCH_CASE(1) MOE_DISPATCH_CASE(2) MOE_DISPATCH_CASE(3) MOE_DISPATCH_CASE(4)
-    MOE_DISPATCH_CASE(5) MOE_DISPATCH_CASE(6) MOE_DISPATCH_CASE(7) MOE_DISPATCH_CASE(8)
-    default: return MOE_ERR_SHAPE;
+  if (counts_ready) {
+    rc = MOE_OK;
+  } else {
+    switch (nw) {
+      MOE_DISPATCH_CASE(1) MOE_DISPATCH_CASE(2) MOE_DISPATCH_CASE(3) MOE_DISPATCH_CASE(4)
+      MOE_DISPATCH_CASE(5) MOE_DISPATCH_CASE(6) MOE_DISPATCH_CASE(7) MOE_DISPATCH_CASE(8)
+      default: return MOE_ERR_SHAPE;
+    }
   }
 #undef MOE_DISPATCH_CASE
   if (rc) return rc;

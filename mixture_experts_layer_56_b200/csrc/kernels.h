@@ -11,18 +11,23 @@ constexpr int kDispatchChunk = 128;  // tokens per dispatch block
 inline int64_t dispatch_num_chunks(int64_t T) { return (T + kDispatchChunk - 1) / kDispatchChunk; }
 int router_num_ctas(int64_t T);
 
+// chunk_counts (nullable): the tensor-core router also writes, per
+// kDispatchChunk tokens, how many chose each expert ([chunks, n]); it returns
+// false in *counted when it did not (the CUDA-core router, or no buffer).
 int launch_router(int dtype, const void* u, const void* E, const float* bias, int64_t T, int d,
                   int n, int K, int flags, int32_t* idx, float* w, float* pstat,
-                  int32_t* status, cudaStream_t st);
+                  int32_t* status, cudaStream_t st, int32_t* chunk_counts = nullptr,
+                  bool* counted = nullptr);
 
 // bf16 router on the tensor cores (router_tc.cu); pstat as launch_router's
 int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T, int d, int n,
                      int K, int flags, int32_t* idx, float* w, float* pstat, int32_t* status,
-                     cudaStream_t st);
+                     int32_t* chunk_counts, cudaStream_t st);
 
+// counts_ready: chunk_counts already hold the per-chunk counts of idx
 int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_counts,
                     int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* perm,
-                    int32_t* inv, cudaStream_t st);
+                    int32_t* inv, cudaStream_t st, bool counts_ready = false);
 
 int launch_gather(int dtype, const void* u, const int32_t* perm, int64_t rows, int d, int K,
                   void* xperm, cudaStream_t st);

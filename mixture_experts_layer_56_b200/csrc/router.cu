@@ -381,10 +381,14 @@ int router_num_ctas(int64_t T) { return static_cast<int>((T + kTokPerCta - 1) / 
 
 int launch_router(int dtype, const void* u, const void* E, const float* bias, int64_t T, int d,
                   int n, int K, int flags, int32_t* idx, float* w, float* pstat,
-                  int32_t* status, cudaStream_t st) {
+                  int32_t* status, cudaStream_t st, int32_t* chunk_counts, bool* counted) {
+  if (counted) *counted = false;
   if (T == 0) return MOE_OK;
-  if (dtype == MOE_DTYPE_BF16 && !(flags & MOE_FLAG_ROUTER_SIMT))
-    return launch_router_tc(u, E, bias, T, d, n, K, flags, idx, w, pstat, status, st);
+  if (dtype == MOE_DTYPE_BF16 && !(flags & MOE_FLAG_ROUTER_SIMT)) {
+    if (counted) *counted = chunk_counts != nullptr;
+    return launch_router_tc(u, E, bias, T, d, n, K, flags, idx, w, pstat, status, chunk_counts,
+                            st);
+  }
   if (dtype == MOE_DTYPE_BF16) {
     if (pstat)
       return launch_router_t<bf16, true>(static_cast<const bf16*>(u), static_cast<const bf16*>(E),

@@ -32,6 +32,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kRtTokens = 128;  // tokens per CTA: one TMEM lane each
+static_assert(kRtTokens == kDispatchChunk, "a router CTA counts exactly one dispatch chunk");
 constexpr int kRtThreads = 128;
 constexpr int kRtBK = 64;  // columns of d per stage (128 bytes of bf16)
 constexpr int kRtMaxStages = 8;
@@ -53,12 +54,14 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmE,
                  const float* __restrict__ bias, int64_t T, int d, int n, int np, int K,
                  int flags, int stages, uint32_t tmem_cols, int32_t* __restrict__ idx,
-                 float* __restrict__ w, float* __restrict__ pstat, int32_t* status) {
+                 float* __restrict__ w, float* __restrict__ pstat, int32_t* status,
+                 int32_t* __restrict__ chunk_counts) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[2 * kRtMaxStages + 2];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ float sbias[256];
+  __shared__ int hist[256];  // this CTA's tokens per expert (chunk_counts)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -97,7 +100,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
     tma_prefetch_desc(&tmE);
   }
   pdl_wait();  // u, E, bias and the outputs belong to earlier stream work
-  for (int e = tid; e < 256; e += kRtThreads) sbias[e] = (bias != nullptr && e < n) ? bias[e] : 0.0f;
+  for (int e = tid; e < 256; e += kRtThreads) {
+    sbias[e] = (bias != nullptr && e < n) ? bias[e] : 0.0f;
+    hist[e] = 0;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -178,6 +184,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
       for (int k = 0; k < K; ++k) {
         idx[t * K + k] = k;
         w[t * K + k] = 0.0f;
+        if (chunk_counts) atomicAdd(&hist[k], 1);
       }
   } else if (NCH == 0) {
     float m = -CUDART_INF_F;
@@ -232,6 +239,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
       if (live) {
         idx[t * K + k] = bi;
         w[t * K + k] = expf(blg - m) * inv_z;
+        if (chunk_counts && bi >= 0) atomicAdd(&hist[bi], 1);
       }
       pv = bv;
       pe = bi;
@@ -349,6 +357,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
       if (live) {
         idx[t * K + k] = e;
         w[t * K + k] = expf((SEL ? l : v) - m) * inv_z;
+        if (chunk_counts && e < n) atomicAdd(&hist[e], 1);
       }
       prev = e;
     }
@@ -360,13 +369,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
   }
+  if (chunk_counts)
+    for (int e = tid; e < n; e += kRtThreads)
+      chunk_counts[static_cast<int64_t>(blockIdx.x) * n + e] = hist[e];
 }
 
 }  // namespace
 
 int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T, int d, int n,
                      int K, int flags, int32_t* idx, float* w, float* pstat, int32_t* status,
-                     cudaStream_t st) {
+                     int32_t* chunk_counts, cudaStream_t st) {
   if (T == 0) return MOE_OK;
   if (d % kRtBK != 0 || n < 1 || n > 256) return MOE_ERR_SHAPE;
   const int np = rt_padded_experts(n);
@@ -391,7 +403,7 @@ int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T,
       attr_done = true;
     }
     return launch_k(kern, grid, kRtThreads, static_cast<size_t>(smem), st, 1, mu, me, bias, T, d,
-                    n, np, K, flags, stages, cols, idx, w, pstat, status);
+                    n, np, K, flags, stages, cols, idx, w, pstat, status, chunk_counts);
   };
   const bool sel = (flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
   const int nch = (np + 31) / 32;
