@@ -5,8 +5,9 @@
 
 A step is one whole layer forward (router, dispatch, expert FFNs, combine)
 over one batch of T synthetic tokens, through the C ABI (moe_layer_forward)
-with the activations resident in HBM.  Between timed steps L2 is flushed (a
-256 MB memset, outside the step's events).  Every rank runs its own batch
+with the activations resident in HBM, replayed from captured CUDA graphs
+(`--eager` launches the kernels directly).  Between timed steps L2 is flushed
+(a 256 MB memset, outside the step's events).  Every rank runs its own batch
 with replicated weights (tokens are independent, so there is no collective on
 the data path: weak scaling); the time is the max over ranks.
 
@@ -14,7 +15,9 @@ One JSON line is printed by rank 0.  Besides the step throughput it holds:
 * e2e: the same metric through moe_layer_forward_host (u and h in pinned
   host memory, both copies inside the timed call);
 * roofline: the grouped gate/up GEMM (the dominant kernel) against the
-  measured dense-bf16 peak, from CUDA events around that kernel;
+  measured dense-bf16 peak (decode-sized batches: the HBM copy peak, for the
+  W1/W3 bytes of the activated experts), from CUDA events around that kernel
+  inside the timed steps;
 * cpu_baseline: the fp64 CPU oracle timed on a bounded sample of tokens;
 * clocks: SM clock and throttle reasons sampled during the timed region.
 `--impl reference` times the CPU oracle alone (the reference arm).
@@ -52,11 +55,15 @@ def workload_desc(wl):
             + (f" Zipf({wl.zipf_s}) router norms" if wl.zipf_s else ""))
 
 
-def weight_bytes_streamed(wl, counts):
-    """Bytes of expert weights a forward must read: every expert hit + shared
-    ones, plus the router centroids (decode roofline)."""
+def weight_bytes_streamed(wl, counts, gate_up_only=False):
+    """Bytes of expert weights a forward must read: every expert hit plus the
+    shared ones (decode roofline).  gate_up_only: the W1/W3 share that the
+    gate/up GEMM reads (2 d I per expert); else all three matrices and the
+    router centroids."""
     el = 2 if wl.dtype == "bf16" else 4
     hit = int((counts > 0).sum())
+    if gate_up_only:
+        return (hit + wl.n_shared) * 2 * wl.d * wl.inter * el
     return (hit + wl.n_shared) * 3 * wl.d * wl.inter * el + wl.n_routed * wl.d * el
 
 
@@ -265,20 +272,38 @@ def run_ours(args):
                             layer.W13_s, layer.W2_s, h, layer.ws,
                             stream=torch.cuda.current_stream(dev))
 
-    graph = None
-    if args.graph:
-        # one forward captured once and replayed per step: the C ABI only
-        # enqueues work on the caller's stream, so it captures as is
+    # CUDA events around the dominant kernel, on the stream it runs on,
+    # inside the timed steps; the other stages are bracketed in a separate
+    # pass so that their events do not stretch the timed steps
+    dominant = L.MOE_KERNEL_GEMM_GATE_UP if wl.dtype == "bf16" else L.MOE_KERNEL_FFN_F32
+    timed_kinds = (dominant,)
+
+    graphs = []
+    if not args.eager:
+        # the forward captured into a few CUDA graphs, replayed in turn, one
+        # per step (the C ABI only enqueues work on the caller's stream, so it
+        # captures as is).  Two of them also capture event records around the
+        # dominant kernel: after the timed loop those events hold the
+        # kernel's last two runs inside the timed steps (the other graphs
+        # carry no events, which would stretch the steps a little).
         forward()
         torch.cuda.synchronize(dev)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            forward()
+        L.moe_profile_read()
+        n_graphs = min(8, max(1, args.steps))
+        for i in range(n_graphs):
+            L.moe_profile_enable(i < 2, kinds=timed_kinds)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                forward()
+            graphs.append(g)
+        L.moe_profile_enable(False)
         torch.cuda.synchronize(dev)
+    step_no = [0]
 
     def step():
-        if graph is not None:
-            graph.replay()
+        if graphs:
+            graphs[step_no[0] % len(graphs)].replay()
+            step_no[0] += 1
         else:
             forward()
 
@@ -295,15 +320,10 @@ def run_ours(args):
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier()
     launches0 = L.moe_launch_count()
-    # CUDA events around the dominant kernel on the launching stream, inside
-    # the timed steps (graph replays carry no events: a separate pass times
-    # those); the other stages are bracketed in a separate pass so that their
-    # events do not stretch the timed steps
-    dominant = L.MOE_KERNEL_GEMM_GATE_UP if wl.dtype == "bf16" else L.MOE_KERNEL_FFN_F32
-    hbm_kinds = (L.MOE_KERNEL_GEMM_GATE_UP, L.MOE_KERNEL_GEMM_DOWN, L.MOE_KERNEL_FFN_F32)
-    timed_kinds = (dominant,) if wl.T >= 1024 and wl.dtype == "bf16" else hbm_kinds
-    L.moe_profile_read()
-    L.moe_profile_enable(graph is None, kinds=timed_kinds)
+    if not graphs:
+        L.moe_profile_read()
+        L.moe_profile_enable(True, kinds=timed_kinds)
+    step_no[0] = 0
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         for i in range(args.steps):
             flush.zero_()
@@ -312,9 +332,9 @@ def run_ours(args):
             ends[i].record(stream)
         barrier()
     launches = L.moe_launch_count() - launches0
-    recs = L.moe_profile_read()
+    recs = L.moe_profile_read()  # eager: every timed step; graphs: each one's last replay
     L.moe_profile_enable(False)
-    if graph is not None:
+    if graphs:
         # replays bypass the library's launch counter: count one eager step
         c0 = L.moe_launch_count()
         forward()
@@ -329,6 +349,7 @@ def run_ours(args):
     tflops = wl.expert_flops() * world * args.steps / (total_ms / 1e3) / 1e12
 
     timed_recs = recs
+    graphs.clear()
     # ---- every stage's device time: a separate, untimed pass ---------------
     L.moe_profile_enable(True)
     for _ in range(20):
@@ -344,10 +365,9 @@ def run_ours(args):
             acc.setdefault(name, []).append(ms)
         return {k: sum(v) / len(v) for k, v in acc.items()}
     stage_ms = mean_ms(stage_recs)
-    # the roofline kernels' time: from the timed steps unless graphs hid them
+    # the roofline kernels' time: from the timed steps
     kernel_ms = dict(stage_ms)
-    if graph is None:
-        kernel_ms.update(mean_ms(timed_recs))
+    kernel_ms.update(mean_ms(timed_recs))
 
     # ---- e2e through the host-buffer entry point ---------------------------
     u_h = u.cpu().pin_memory()
@@ -379,17 +399,20 @@ def run_ours(args):
                     "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)",
                     "flops_per_launch": gate_up_flops, "ms_per_launch": ms}
     else:
+        # decode-sized batches: the gate/up GEMM streams the activated experts'
+        # W1/W3 (the fp32 layer's single FFN kernel streams all three)
         counts = routed_counts(layer, u, L, torch)
-        byts = weight_bytes_streamed(wl, counts)
-        gemm_ms = sum(kernel_ms.get(k, 0.0) for k in ("grouped_gemm_gate_up_swiglu",
-                                                      "grouped_gemm_down", "ffn_f32"))
-        achieved = byts / (gemm_ms / 1e3) / 1e9 if gemm_ms > 0 else None
+        bf16 = wl.dtype == "bf16"
+        byts = weight_bytes_streamed(wl, counts, gate_up_only=bf16)
+        name = "grouped_gemm_gate_up_swiglu" if bf16 else "ffn_f32"
+        ms = kernel_ms.get(name, 0.0)
+        achieved = byts / (ms / 1e3) / 1e9 if ms > 0 else None
         peak = float(peaks["hbm_gbs"])
-        roofline = {"bound": "hbm", "kernel": "expert GEMMs (gate/up + down)",
+        roofline = {"bound": "hbm", "kernel": name,
                     "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": (achieved / peak) if achieved else None, "traffic": None,
                     "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json)",
-                    "bytes_per_step": byts}
+                    "bytes_per_launch": byts, "ms_per_launch": ms}
 
     # ---- CPU baseline (rank 0, N = 1 only) -----------------------------------
     cpu = None
@@ -407,7 +430,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic",
             "config": {"workload": workload_desc(wl), "tokens_per_gpu_step": wl.T,
-                       "gemm_tiles": args.gemm, "cuda_graph": bool(args.graph),
+                       "gemm_tiles": args.gemm, "cuda_graph": not args.eager,
                        "parallelism": f"replicas x{world} (token batches, no collective)",
                        "l2": "flushed between steps (256 MB memset outside the step events)",
                        "init": "seeded splitmix64/Box-Muller normals, bf16"},
@@ -455,8 +478,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--graph", action="store_true",
-                    help="replay each step from a captured CUDA graph")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every step's kernels directly instead of replaying a captured "
+                         "CUDA graph")
     ap.add_argument("--gemm", default="auto", choices=["auto", "single", "pair"],
                     help="tile shape of the expert GEMMs (default: chosen by the library)")
     args = ap.parse_args()

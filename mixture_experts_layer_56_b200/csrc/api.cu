@@ -49,6 +49,17 @@ Profiler& prof() {
 }
 constexpr size_t kMaxProfRecs = 4096;
 
+// Records `e` on `st`; inside a stream capture as an event node of the graph
+// (a plain record there is only a dependency within the capture), so that
+// every replay records it.
+void record_event(cudaEvent_t e, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, st);
+}
+
 // RAII bracket: records the start event now and the end event when it goes
 // out of scope (after the stage's launches were enqueued).
 class Stage {
@@ -60,7 +71,7 @@ class Stage {
     if (p.recs.size() >= kMaxProfRecs) return;
     ProfRec r{kind, p.get(), p.get()};
     if (!r.beg || !r.end) return;
-    cudaEventRecord(r.beg, st_);
+    record_event(r.beg, st_);
     p.recs.push_back(r);
     idx_ = static_cast<long>(p.recs.size()) - 1;
   }
@@ -68,7 +79,7 @@ class Stage {
     if (idx_ < 0) return;
     Profiler& p = prof();
     std::lock_guard<std::mutex> lock(p.mu);
-    cudaEventRecord(p.recs[static_cast<size_t>(idx_)].end, st_);
+    record_event(p.recs[static_cast<size_t>(idx_)].end, st_);
   }
 
  private:
@@ -404,8 +415,10 @@ int moe_profile_read(int32_t* kinds, float* ms, int32_t max, int32_t* count) {
     if (n < max) {
       float t = 0.0f;
       if (cudaEventSynchronize(r.end) != cudaSuccess ||
-          cudaEventElapsedTime(&t, r.beg, r.end) != cudaSuccess)
+          cudaEventElapsedTime(&t, r.beg, r.end) != cudaSuccess) {
         rc = MOE_ERR_CUDA;
+        cudaGetLastError();  // a failed query must not surface in a later launch check
+      }
       kinds[n] = r.kind;
       ms[n] = t;
       ++n;
