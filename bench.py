@@ -388,15 +388,20 @@ def run_ours(args):
 
     # ---- roofline of the dominant kernel -----------------------------------
     peaks, peak_src = load_peaks()
+    clocks = clk.summary()
     if wl.dtype == "bf16" and "grouped_gemm_gate_up_swiglu" in kernel_ms and wl.T >= 1024:
         gate_up_flops = 4.0 * wl.T * (wl.top_k + wl.n_shared) * wl.d * wl.inter
         ms = kernel_ms["grouped_gemm_gate_up_swiglu"]
         achieved = gate_up_flops / (ms / 1e3) / 1e12
-        peak = float(peaks["bf16_tflops"])
+        # the sustained GEMM peak when the power cap held the clocks down
+        # during the timed steps, else the burst one
+        capped = "sw_power_cap" in (clocks.get("reasons") or [])
+        peak = float(peaks["bf16_tflops_sustained" if capped else "bf16_tflops"])
         roofline = {"bound": "tensor", "kernel": "grouped_gemm_gate_up_swiglu",
                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": ncu_traffic(wl.name),
-                    "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)",
+                    "peak_source": f"{peak_src} bf16 {'sustained' if capped else 'burst'} "
+                                   f"(MEASURED_PEAKS.json)",
                     "flops_per_launch": gate_up_flops, "ms_per_launch": ms}
     else:
         # decode-sized batches: the gate/up GEMM streams the activated experts'
@@ -423,7 +428,6 @@ def run_ours(args):
                          f"({dt:.1f} s)"}
 
     if rank == 0:
-        clocks = clk.summary()
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,

@@ -230,3 +230,40 @@ def test_balance_statistics_every_router_variant(n):
     f_ref, P_ref, _ = O.expert_balance(s, rep["gpu"]["idx"])
     np.testing.assert_allclose(to_numpy(f), f_ref, rtol=1e-6)
     np.testing.assert_allclose(to_numpy(Pm), P_ref, rtol=1e-4, atol=1e-7)
+
+
+def test_forward_replays_from_a_cuda_graph_bitwise():
+    """moe_layer_forward only enqueues work on the caller's stream: captured
+    into a CUDA graph (its kernels keep programmatic dependent launch), each
+    replay gives the eager result bit for bit, also after the input changes."""
+    wl = W("graph", T=600, d=256, n_routed=24, n_shared=1, inter=128, top_k=4)
+    x = S.make_inputs(wl)
+    layer = MoELayer(x)
+    u = to_device(x.u, "cuda:0")
+    h = torch.empty_like(u)
+
+    def fwd():
+        L.moe_layer_forward(layer.shape, u, layer.E, layer.bias, layer.W13, layer.W2,
+                            layer.W13_s, layer.W2_s, h, layer.ws,
+                            stream=torch.cuda.current_stream())
+
+    fwd()
+    torch.cuda.synchronize()
+    ref = to_numpy(h).copy()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd()
+    for _ in range(3):
+        h.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(to_numpy(h), ref)
+    u.copy_(torch.flip(u, dims=[0]))  # new tokens in the same buffer
+    g.replay()
+    torch.cuda.synchronize()
+    ref2 = to_numpy(h).copy()
+    fwd()
+    torch.cuda.synchronize()
+    assert np.array_equal(to_numpy(h), ref2)
+    assert not np.array_equal(ref, ref2)
+    assert layer.status() == 0
