@@ -35,6 +35,13 @@
  *   the workspace's status word, read with moe_read_status.
  * - Results are bitwise reproducible from run to run (no atomics decide any
  *   value or order).
+ * - Kernels are launched with programmatic dependent launch: one may start
+ *   its set-up while the previous kernel on the stream finishes, but it reads
+ *   and writes no global memory before that kernel has completed, so the
+ *   usual stream order holds for the caller's own work too.
+ * - moe_layer_forward only enqueues kernels on `stream` (no allocation, no
+ *   host synchronisation), so a caller may capture it into a CUDA graph and
+ *   replay it; replays give the eager result bit for bit.
  */
 #ifndef MOE_H_
 #define MOE_H_
@@ -215,7 +222,7 @@ int moe_expert_balance(const moe_shape_t* shape, const void* u, const void* E,
 int moe_read_status(const void* ws, int32_t* status, moe_stream_t stream);
 
 /* Tracing: device time of each stage.  While enabled, every kernel (the
-   three dispatch kernels count as one stage) that libmoe launches is
+   dispatch kernels count as one stage) that libmoe launches is
    bracketed by CUDA events recorded on its stream.  moe_profile_read waits
    for those events and returns, oldest first, the stage kind (MOE_KERNEL_*)
    and elapsed milliseconds of each bracketed launch since the last read:

@@ -1,6 +1,8 @@
 // Router of the DeepSeekMoE layer (§3.2, eqs. (10)-(11)): fp32 logits
 // l_{t,i} = sum_j u_{t,j} e_{i,j} (+ b_i) on CUDA cores, softmax over the
-// routed experts and top-K selection with warp shuffles.
+// routed experts and top-K selection with warp shuffles.  It serves the fp32
+// layer and, with MOE_FLAG_ROUTER_SIMT, bf16; bf16 routes on the tensor cores
+// by default (router_tc.cu), and launch_router below picks between them.
 //
 // A CTA owns 32 tokens and all experts.  A producer warp streams 128-byte
 // column slices of u (32 rows) and E (NP rows) into a 4-stage shared-memory
