@@ -282,16 +282,16 @@ def run_ours(args):
     if not args.eager:
         # the forward captured into a few CUDA graphs, replayed in turn, one
         # per step (the C ABI only enqueues work on the caller's stream, so it
-        # captures as is).  Two of them also capture event records around the
-        # dominant kernel: after the timed loop those events hold the
-        # kernel's last two runs inside the timed steps (the other graphs
-        # carry no events, which would stretch the steps a little).
+        # captures as is).  Half of them also capture event records around
+        # the dominant kernel: after the timed loop those events hold the
+        # kernel's last runs inside the timed steps (the other graphs carry
+        # no events, which would stretch the steps a little).
         forward()
         torch.cuda.synchronize(dev)
         L.moe_profile_read()
         n_graphs = min(8, max(1, args.steps))
         for i in range(n_graphs):
-            L.moe_profile_enable(i < 2, kinds=timed_kinds)
+            L.moe_profile_enable(i % 2 == 0, kinds=timed_kinds)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 forward()

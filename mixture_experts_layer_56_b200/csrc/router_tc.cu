@@ -39,6 +39,32 @@ constexpr int kRtMaxStages = 8;
 constexpr int kRtSmemBudget = 200 * 1024;
 constexpr int kRtTileBytes = kRtTokens * kRtBK * 2;
 
+// 32 consecutive fp32 columns of this thread's TMEM lane from registers
+// (shape 32x32b, x32); tmem_st_wait() before the columns are read back
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+      ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// 16 bytes / 4 bytes of a cluster peer's shared memory (mapa address)
+__device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_shared_cluster_s32(uint32_t cluster_addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
 inline int rt_padded_experts(int n) { return (n + 15) / 16 * 16; }
 inline int rt_stage_bytes(int np) { return kRtTileBytes + np * kRtBK * 2; }
 inline int rt_stages(int np) {
@@ -48,8 +74,10 @@ inline int rt_stages(int np) {
 
 // NCH > 0: a token's logits (NCH chunks of 32) stay in registers after one
 // TMEM read, SEL = the bias only steers the selection.  NCH = 0: any expert
-// count; the chunks are re-read from TMEM for every pass.
-template <bool STATS, int NCH, bool SEL>
+// count; the chunks are re-read from TMEM for every pass.  CS > 1: a cluster
+// of CS CTAs shares one 128-token tile, rank r computing the logits over
+// its share of d; rank 0 adds the partials in rank order and selects.
+template <bool STATS, int NCH, bool SEL, int CS>
 __global__ void __launch_bounds__(kRtThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmE,
                  const float* __restrict__ bias, int64_t T, int d, int n, int np, int K,
@@ -76,8 +104,12 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int m0 = static_cast<int>(blockIdx.x) * kRtTokens;
-  const int nkb = d / kRtBK;
+  const int tile = static_cast<int>(blockIdx.x) / CS;
+  const int m0 = tile * kRtTokens;
+  const int crank = CS > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int nkb_all = d / kRtBK;
+  const int kb0 = crank * nkb_all / CS, kb1 = (crank + 1) * nkb_all / CS;
+  const int nkb = kb1 - kb0;
   volatile int* abort_p = &abort_flag;
 
   if (tid == 0) {
@@ -116,12 +148,12 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_parity = 0;
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int i = 0; i < nkb; ++i) {
         if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_p, status)) { ok = false; break; }
         const uint32_t sa = smem_base + stage * stage_bytes;
         mbar_arrive_expect_tx(full_bar(stage), stage_bytes);
-        tma_load_2d(sa, &tmU, full_bar(stage), kb * kRtBK, m0);
-        tma_load_2d(sa + kRtTileBytes, &tmE, full_bar(stage), kb * kRtBK, 0);
+        tma_load_2d(sa, &tmU, full_bar(stage), (kb0 + i) * kRtBK, m0);
+        tma_load_2d(sa + kRtTileBytes, &tmE, full_bar(stage), (kb0 + i) * kRtBK, 0);
         issued |= 1u << stage;
         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == stages) { stage = 0; phase ^= 1u; }
@@ -168,7 +200,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
 
   // ------------------------------------------------ softmax and top-K ------
   pdl_trigger();
-  const bool got = __all_sync(0xffffffffu, wait_bounded(done_bar, 0, abort_p, status) ? 1 : 0);
+  bool got = __all_sync(0xffffffffu, wait_bounded(done_bar, 0, abort_p, status) ? 1 : 0);
   tc_fence_after();
   const int r = warp * 32 + lane;
   const int64_t t = static_cast<int64_t>(m0) + r;
@@ -176,8 +208,64 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
   const uint32_t trow = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
   const int nch = (np + 31) / 32;
   const bool select_only = (flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
+  bool selects = true;  // this CTA runs the softmax and selection
 
-  if (!got) {
+  if constexpr (CS > 1) {
+    // Each rank's partial logits go to its own shared memory (the ring is
+    // free: every MMA that read it has completed).  Rank 0 adds the ranks'
+    // partials in rank order and writes the sums into its TMEM, where the
+    // selection below reads them.  Every CTA reaches both cluster barriers.
+    // Only rows of real tokens move (one row at T = 1).
+    __shared__ int got_flag;
+    const int ldp = nch * 32 + 4;
+    float* part = reinterpret_cast<float*>(smem);
+    const bool warp_live = __any_sync(0xffffffffu, live);
+    if (got && warp_live) {
+      for (int c = 0; c < nch; ++c) {
+        float x[32];
+        tmem_ld32(trow + c * 32, x);
+        tmem_ld_wait_regs(x);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(part + r * ldp + c * 32 + j) =
+              make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+      }
+    }
+    const bool cta_got = __syncthreads_and(got ? 1 : 0) != 0;
+    if (tid == 0) got_flag = cta_got ? 1 : 0;
+    cluster_sync_all();
+    if (crank == 0) {
+      int all = 1;
+      for (int rk = 0; rk < CS; ++rk) all &= ld_shared_cluster_s32(map_to_cta(smem_addr(&got_flag), rk));
+      got = all != 0;
+      if (got && warp_live) {
+        for (int c = 0; c < nch; ++c) {
+          float x[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) x[j] = 0.0f;
+          for (int rk = 0; rk < (live ? CS : 0); ++rk) {
+            const uint32_t row = map_to_cta(smem_addr(part + r * ldp + c * 32), rk);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 v = ld_shared_cluster_v4(row + j * 4);
+              x[j] += v.x;
+              x[j + 1] += v.y;
+              x[j + 2] += v.z;
+              x[j + 3] += v.w;
+            }
+          }
+          tmem_st32(trow + c * 32, x);
+        }
+        tmem_st_wait();
+      }
+    }
+    cluster_sync_all();  // the peers' partials stay until rank 0 has read them
+    selects = crank == 0;
+  }
+
+  if (!selects) {
+    // a peer rank: its share of the logits is with rank 0
+  } else if (!got) {
     // results stay in range for the stages downstream; the status word says
     // that they are not to be used
     if (live)
@@ -264,7 +352,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
         }
       }
       __syncwarp();
-      const int64_t g = static_cast<int64_t>(blockIdx.x) * (kRtTokens / 32) + warp;
+      const int64_t g = static_cast<int64_t>(tile) * (kRtTokens / 32) + warp;
       if (g * 32 < T) {
         for (int e = lane; e < n; e += 32) {
           float a = 0.0f;
@@ -309,7 +397,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
       for (int j = 0; j < NR; ++j)
         if (j < np) sc[lane * ld + j] = (live && j < n) ? expf((SEL ? lg[j] : key[j]) - m) / z : 0.0f;
       __syncwarp();
-      const int64_t g = static_cast<int64_t>(blockIdx.x) * (kRtTokens / 32) + warp;
+      const int64_t g = static_cast<int64_t>(tile) * (kRtTokens / 32) + warp;
       if (g * 32 < T) {
         for (int e = lane; e < n; e += 32) {
           float a = 0.0f;
@@ -369,9 +457,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
   }
-  if (chunk_counts)
+  if (chunk_counts && crank == 0)
     for (int e = tid; e < n; e += kRtThreads)
-      chunk_counts[static_cast<int64_t>(blockIdx.x) * n + e] = hist[e];
+      chunk_counts[static_cast<int64_t>(tile) * n + e] = hist[e];
 }
 
 }  // namespace
@@ -393,8 +481,18 @@ int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T,
                    static_cast<uint64_t>(n), static_cast<uint64_t>(d) * 2, kRtBK,
                    static_cast<uint32_t>(np)))
     return MOE_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>((T + kRtTokens - 1) / kRtTokens);
-  auto go = [&](auto kern, bool& attr_done) -> int {
+  const int64_t tiles = (T + kRtTokens - 1) / kRtTokens;
+  // few tiles: split d over a cluster so that more SMs stream u and E
+  static int sm_count[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  if (sm_count[dev] == 0 &&
+      cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int cs = 1;
+  if (!pstat)
+    while (cs < 8 && tiles * cs * 2 <= sm_count[dev] && d / kRtBK >= 2 * cs) cs *= 2;
+  auto go = [&](auto kern, bool& attr_done, unsigned cl) -> int {
     // one opt-in size covering every expert count (smem never exceeds it)
     if (!attr_done) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -402,18 +500,22 @@ int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T,
         return MOE_ERR_CUDA;
       attr_done = true;
     }
-    return launch_k(kern, grid, kRtThreads, static_cast<size_t>(smem), st, 1, mu, me, bias, T, d,
-                    n, np, K, flags, stages, cols, idx, w, pstat, status, chunk_counts);
+    return launch_k(kern, dim3(static_cast<unsigned>(tiles) * cl), kRtThreads,
+                    static_cast<size_t>(smem), st, cl, mu, me, bias, T, d, n, np, K, flags, stages,
+                    cols, idx, w, pstat, status, chunk_counts);
   };
   const bool sel = (flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
   const int nch = (np + 31) / 32;
   // register-resident variants up to 64 experts (128 without SEL)
   // (with statistics, beyond 64 experts the register variant would spill)
   const int v = (nch <= 2 || (nch <= 4 && !sel && !pstat)) ? nch : 0;
-#define MOE_RT_GO(STATS, NCH, SEL)                                  \
-  {                                                                 \
-    static bool done = false;                                       \
-    return go(router_tc_kernel<STATS, NCH, SEL>, done);             \
+#define MOE_RT_GO(STATS, NCH, SEL)                                                   \
+  {                                                                                  \
+    static bool done1 = false, done2 = false, done4 = false, done8 = false;          \
+    if (STATS || cs == 1) return go(router_tc_kernel<STATS, NCH, SEL, 1>, done1, 1u); \
+    if (cs == 2) return go(router_tc_kernel<STATS, NCH, SEL, (STATS ? 1 : 2)>, done2, 2u); \
+    if (cs == 4) return go(router_tc_kernel<STATS, NCH, SEL, (STATS ? 1 : 4)>, done4, 4u); \
+    return go(router_tc_kernel<STATS, NCH, SEL, (STATS ? 1 : 8)>, done8, 8u);        \
   }
 #define MOE_RT_VARIANTS(STATS)                                      \
   if (v == 1 && sel) MOE_RT_GO(STATS, 1, true)                      \
