@@ -482,7 +482,9 @@ int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T,
                    static_cast<uint32_t>(np)))
     return MOE_ERR_CUDA;
   const int64_t tiles = (T + kRtTokens - 1) / kRtTokens;
-  // few tiles: split d over a cluster so that more SMs stream u and E
+  // few tiles (short batches): split d over a cluster so that more SMs
+  // stream u and E; with many tiles every SM is busy and the exchange of
+  // partial logits would only add work
   static int sm_count[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
@@ -490,7 +492,7 @@ int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T,
       cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return MOE_ERR_CUDA;
   int cs = 1;
-  if (!pstat)
+  if (!pstat && tiles <= 16)
     while (cs < 8 && tiles * cs * 2 <= sm_count[dev] && d / kRtBK >= 2 * cs) cs *= 2;
   auto go = [&](auto kern, bool& attr_done, unsigned cl) -> int {
     // one opt-in size covering every expert count (smem never exceeds it)
