@@ -165,11 +165,14 @@ def test_simt_router_full(wl):
 
 # expert counts that reach every epilogue variant of the tensor-core router:
 # 1, 2, 3 and 4 register chunks, and the chunked path (256 experts, or
-# select-only bias beyond 64 experts)
+# select-only bias beyond 64 experts), with and without the cluster split
 ROUTER_CASES = CASES + [
     W("router_90", T=300, d=256, n_routed=90, n_shared=1, inter=64, top_k=6, bias_var=0.5),
     W("router_128", T=300, d=256, n_routed=128, n_shared=1, inter=64, top_k=12),
     W("router_256", T=300, d=256, n_routed=256, n_shared=1, inter=64, top_k=8),
+    # more than 16 tiles of 128 tokens: one CTA per tile (no cluster split)
+    W("router_t2200_n40", T=2200, d=256, n_routed=40, n_shared=1, inter=64, top_k=5),
+    W("router_t2200_n256", T=2200, d=256, n_routed=256, n_shared=1, inter=64, top_k=8),
 ]
 ROUTER_FLAGS = {"bias_in_softmax": 0, "bias_select_only": L.MOE_FLAG_BIAS_SELECT_ONLY}
 
