@@ -189,22 +189,24 @@ dispatch_scatter_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n
 }
 
 // The whole dispatch in one block, for batches of at most kDispatchChunk
-// tokens (decode): counts, the scan over experts and the scatter.
+// tokens (decode): counts, the scan over experts and the scatter.  Each warp
+// visits only the experts its own tokens chose (a handful at decode sizes).
 template <int NW, int KMAX>
 __global__ void __launch_bounds__(kDispThreads)
 dispatch_single_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n,
                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                        int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
   __shared__ int wc[kDispWarps][256];
+  __shared__ int tot[256];
   pdl_wait();
   pdl_trigger();
-  __shared__ int tot[256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = threadIdx.x;
+  for (int i = threadIdx.x; i < kDispWarps * 256; i += blockDim.x) (&wc[0][0])[i] = 0;
   int ek[KMAX];
 #pragma unroll
   for (int k = 0; k < KMAX; ++k) ek[k] = (t < T && k < K) ? idx[t * K + k] : -1;
-  uint32_t mask[NW];
+  uint32_t mask[NW], um[NW];
 #pragma unroll
   for (int w = 0; w < NW; ++w) mask[w] = 0;
 #pragma unroll
@@ -212,9 +214,19 @@ dispatch_single_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n,
 #pragma unroll
     for (int w = 0; w < NW; ++w)
       if (ek[k] >= 0 && (ek[k] >> 5) == w) mask[w] |= 1u << (ek[k] & 31);
-  warp_counts<NW>(mask, n, warp, lane, wc);
+#pragma unroll
+  for (int w = 0; w < NW; ++w) um[w] = __reduce_or_sync(kFull, mask[w]);
+  __syncthreads();  // wc is zero
+  // wc[warp][e] = this warp's tokens that chose e
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    for (uint32_t m = um[w]; m != 0; m &= m - 1) {
+      const int b = __ffs(m) - 1;
+      const unsigned bal = __ballot_sync(kFull, (mask[w] >> b) & 1u);
+      if (lane == 0) wc[warp][w * 32 + b] = __popc(bal);
+    }
+  }
   __syncthreads();
-  // per-expert totals (two experts per thread), then an exclusive scan
   for (int e = threadIdx.x; e < 256; e += blockDim.x) {
     int c = 0;
     if (e < n)
@@ -223,15 +235,29 @@ dispatch_single_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n,
     if (e < n) counts[e] = c;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int e = 0; e < n; ++e) {
-      const int c = tot[e];
-      tot[e] = run;
-      offsets[e] = run;
-      run += c;
+  // exclusive scan over the experts: one warp, eight entries a lane
+  if (warp == 0) {
+    int v[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = tot[lane * 8 + i];
+      sum += v[i];
     }
-    offsets[n] = run;
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane * 8 + i;
+      tot[e] = run;
+      if (e < n) offsets[e] = run;
+      run += v[i];
+    }
+    if (lane == 31) offsets[n] = incl;
   }
   __syncthreads();
   for (int e = threadIdx.x; e < n; e += blockDim.x) {
@@ -246,9 +272,9 @@ dispatch_single_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n,
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
   for (int w = 0; w < NW; ++w) {
-    for (int b = 0; b < 32; ++b) {
+    for (uint32_t m = um[w]; m != 0; m &= m - 1) {
+      const int b = __ffs(m) - 1;
       const int e = w * 32 + b;
-      if (e >= n) break;
       const bool has = (mask[w] >> b) & 1u;
       const unsigned bal = __ballot_sync(kFull, has);
       if (has) {
