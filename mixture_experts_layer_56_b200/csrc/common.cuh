@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -88,6 +90,21 @@ __device__ __forceinline__ void pdl_trigger() {
 // ---------------------------------------------------------------------------
 void count_launch(int n = 1);
 int check_launch();  // MOE_OK or MOE_ERR_CUDA after a <<<>>> launch
+
+// A kernel's opt-in dynamic shared-memory size, set on the current device
+// the first time it launches there (the attribute belongs to the device's
+// copy of the kernel; `done` holds one bit per device).
+inline int ensure_smem_optin(const void* kern, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return MOE_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  done.fetch_or(bit, std::memory_order_release);
+  return MOE_OK;
+}
 
 // Launch with programmatic stream serialisation (the kernel must call
 // pdl_wait() before touching global memory) and, if cluster > 1, thread

@@ -391,14 +391,10 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, 
 template <int BN, int EPI>
 static int launch_impl(const GemmMaps& m, const GroupedGemmArgs& args, int grid,
                        cudaStream_t stream) {
-  static bool attr_done = false;  // set once per instantiation (per process)
+  static std::atomic<uint64_t> optin{0};
   auto kern = grouped_gemm_kernel<BN, EPI>;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem_bytes<BN>()) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    attr_done = true;
-  }
+  if (int rc = ensure_smem_optin(reinterpret_cast<const void*>(kern), smem_bytes<BN>(), optin))
+    return rc;
   return launch_k(kern, grid, kThreads, smem_bytes<BN>(), stream, 1, m.a_r, m.a_s, m.b_r, m.b_s,
                   args);
 }

@@ -419,14 +419,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
 template <int BN, int EPI>
 int launch_pair_impl(const GemmMaps& m, const GroupedGemmArgs& args, int clusters,
                      cudaStream_t stream) {
-  static bool attr_done = false;
+  static std::atomic<uint64_t> optin{0};
   auto kern = grouped_gemm_pair_kernel<BN, EPI>;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             pair_smem_bytes<BN, EPI>()) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    attr_done = true;
-  }
+  if (int rc = ensure_smem_optin(reinterpret_cast<const void*>(kern), pair_smem_bytes<BN, EPI>(),
+                                 optin))
+    return rc;
   return launch_k(kern, dim3(2 * clusters), kPairThreads, pair_smem_bytes<BN, EPI>(), stream, 2,
                   m.a_r, m.a_s, m.b_r, m.b_s, args);
 }

@@ -494,14 +494,10 @@ int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T,
   int cs = 1;
   if (!pstat && tiles <= 16)
     while (cs < 8 && tiles * cs * 2 <= sm_count[dev] && d / kRtBK >= 2 * cs) cs *= 2;
-  auto go = [&](auto kern, bool& attr_done, unsigned cl) -> int {
+  auto go = [&](auto kern, std::atomic<uint64_t>& optin, unsigned cl) -> int {
     // one opt-in size covering every expert count (smem never exceeds it)
-    if (!attr_done) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kRtSmemBudget + 1024) != cudaSuccess)
-        return MOE_ERR_CUDA;
-      attr_done = true;
-    }
+    if (int rc = ensure_smem_optin(reinterpret_cast<const void*>(kern), kRtSmemBudget + 1024, optin))
+      return rc;
     return launch_k(kern, dim3(static_cast<unsigned>(tiles) * cl), kRtThreads,
                     static_cast<size_t>(smem), st, cl, mu, me, bias, T, d, n, np, K, flags, stages,
                     cols, idx, w, pstat, status, chunk_counts);
@@ -513,7 +509,7 @@ int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T,
   const int v = (nch <= 2 || (nch <= 4 && !sel && !pstat)) ? nch : 0;
 #define MOE_RT_GO(STATS, NCH, SEL)                                                   \
   {                                                                                  \
-    static bool done1 = false, done2 = false, done4 = false, done8 = false;          \
+    static std::atomic<uint64_t> done1{0}, done2{0}, done4{0}, done8{0};            \
     if (STATS || cs == 1) return go(router_tc_kernel<STATS, NCH, SEL, 1>, done1, 1u); \
     if (cs == 2) return go(router_tc_kernel<STATS, NCH, SEL, (STATS ? 1 : 2)>, done2, 2u); \
     if (cs == 4) return go(router_tc_kernel<STATS, NCH, SEL, (STATS ? 1 : 4)>, done4, 4u); \
