@@ -400,6 +400,8 @@ def run_ours(args):
         roofline = {"bound": "tensor", "kernel": "grouped_gemm_gate_up_swiglu",
                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": ncu_traffic(wl.name),
+                    "frac_of_burst": achieved / float(peaks["bf16_tflops"]),
+                    "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"]),
                     "peak_source": f"{peak_src} bf16 {'sustained' if capped else 'burst'} "
                                    f"(MEASURED_PEAKS.json)",
                     "flops_per_launch": gate_up_flops, "ms_per_launch": ms}

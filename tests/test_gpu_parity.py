@@ -270,3 +270,11 @@ def test_forward_replays_from_a_cuda_graph_bitwise():
     assert np.array_equal(to_numpy(h), ref2)
     assert not np.array_equal(ref, ref2)
     assert layer.status() == 0
+
+
+def test_half_activated_small_shapes():
+    """Half-activated variant (§4.5, Figs. 5-6): the small layer's shapes with about half
+    the routed experts per token (K = 3 instead of 7), same kernels."""
+    wl = W("half_activated", T=1500, d=1280, n_routed=63, n_shared=1, inter=896, top_k=3)
+    rep = P.full_parity(S.make_inputs(wl))
+    assert rep["gpu"]["counts"].sum() == 1500 * 3
