@@ -170,6 +170,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   const int total_tiles = tile_start[G];
+  const int n_long = (hs && args.kb_shared > args.kb_routed) ? tile_start[1] : 0;
+  const int workers = static_cast<int>(gridDim.x);
 
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer ----
@@ -187,7 +189,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
       uint32_t issued = 0, issued_parity = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+        const TileInfo ti = decode_tile(place_tile(tile, total_tiles, workers, n_long), tile_start, G, hs,
+                                        args.nt_routed, args.nt_shared);
         const CUtensorMap* ma = ti.shared ? &tmA_s : &tmA_r;
         const CUtensorMap* mb = ti.shared ? &tmB_s : &tmB_r;
         const int row = grp_row0[ti.g] + ti.m_blk * BM;
@@ -232,7 +235,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++it) {
-        const TileInfo ti = decode_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+        const TileInfo ti = decode_tile(place_tile(tile, total_tiles, workers, n_long), tile_start, G, hs,
+                                        args.nt_routed, args.nt_shared);
         const int nkb = ti.shared ? args.kb_shared : args.kb_routed;
         const int acc = it & 1;
         const uint32_t ap = (it >> 1) & 1;
@@ -269,7 +273,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
     const int r = q * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+      const TileInfo ti = decode_tile(place_tile(tile, total_tiles, workers, n_long), tile_start, G, hs,
+                                        args.nt_routed, args.nt_shared);
       const int acc = it & 1;
       const uint32_t ap = (it >> 1) & 1;
       if (!wait_bounded(tfull_bar(acc), ap, abort_p, args.status)) break;

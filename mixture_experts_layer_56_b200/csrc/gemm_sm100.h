@@ -34,6 +34,22 @@ struct GroupedGemmArgs {
   int32_t a_rows;
 };
 
+// Tile placement of the persistent GEMMs.  Worker w (a CTA, or a CTA pair)
+// takes positions w, w + workers, ...; position v computes tile
+// place_tile(v, ...).  Tiles are numbered with the shared-expert group first,
+// and its n_long tiles may be longer (the down GEMM's K is K_s * I there).
+// With three or more positions per worker the long tiles stay first (they
+// start early).  With at most two, they go to the last positions of the
+// workers that get one position fewer, so that no worker adds a long tile
+// to a full share of short ones.
+__device__ __forceinline__ int place_tile(int v, int total, int workers, int n_long) {
+  const int q = total / workers, r = total - q * workers;
+  if (n_long == 0 || q < 1 || q > 2 || n_long > workers - r) return v;
+  const int p0 = (q - 1) * workers + r;  // first position of a short worker's last round
+  if (v >= p0 && v < p0 + n_long) return v - p0;
+  return v < p0 ? v + n_long : v;
+}
+
 // A maps: rank 2 {K, rows}; B maps: rank 3 {K, N rows, experts}; bf16, box
 // {64, 128 (A) or BN (B)}, 128-byte swizzle.
 struct GemmMaps {

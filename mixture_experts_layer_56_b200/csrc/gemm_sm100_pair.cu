@@ -206,6 +206,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   const int total_tiles = tile_start[G];
+  const int n_long = (hs && args.kb_shared > args.kb_routed) ? tile_start[1] : 0;
 
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer ----
@@ -221,7 +222,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       bool ok = true;
       for (int tile = cluster; tile < total_tiles && ok; tile += nclusters) {
         const PairTile ti =
-            decode_pair_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+            decode_pair_tile(place_tile(tile, total_tiles, nclusters, n_long), tile_start, G, hs,
+                             args.nt_routed, args.nt_shared);
         const CUtensorMap* ma = ti.shared ? &tmA_s : &tmA_r;
         const CUtensorMap* mb = ti.shared ? &tmB_s : &tmB_r;
         const int row = grp_row0[ti.g] + ti.m_blk * PBM + static_cast<int>(rank) * HBM_ROWS;
@@ -261,7 +263,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       bool ok = true;
       for (int tile = cluster; tile < total_tiles && ok; tile += nclusters, ++it) {
         const PairTile ti =
-            decode_pair_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+            decode_pair_tile(place_tile(tile, total_tiles, nclusters, n_long), tile_start, G, hs,
+                             args.nt_routed, args.nt_shared);
         const int nkb = ti.shared ? args.kb_shared : args.kb_routed;
         const int acc = it & 1;
         const uint32_t ap = (it >> 1) & 1;
@@ -301,7 +304,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
     int it = 0;
     for (int tile = cluster; tile < total_tiles; tile += nclusters, ++it) {
       const PairTile ti =
-          decode_pair_tile(tile, tile_start, G, hs, args.nt_routed, args.nt_shared);
+          decode_pair_tile(place_tile(tile, total_tiles, nclusters, n_long), tile_start, G, hs,
+                             args.nt_routed, args.nt_shared);
       const int acc = it & 1;
       const uint32_t ap = (it >> 1) & 1;
       if (!wait_bounded(tfull_bar(acc), ap, abort_p, args.status)) break;
