@@ -59,3 +59,22 @@ def test_pins_reject_planted_mistake(name, golden_dir, monkeypatch):
     monkeypatch.setitem(O.__dict__, "_orig_combine", O.combine)
     monkeypatch.setattr(O, attr, fn)
     assert not _worked_example_passes(golden_dir), name
+
+
+def test_routed_rows_pin_rejects_a_wrong_token_of_a_slot(monkeypatch):
+    """Planted mistake: a position's token taken as slot % K instead of
+    slot // K (the slot is t*K + k)."""
+    from tests.test_oracle_pins import test_routed_expert_outputs_against_torch as pin
+
+    def wrong(u, perm, offsets, K, W1, W3, W2):
+        y = np.zeros((perm.size, u.shape[1]))
+        for e in range(W1.shape[0]):
+            lo, hi = int(offsets[e]), int(offsets[e + 1])
+            if hi > lo:
+                y[lo:hi] = O.swiglu_ffn(u[perm[lo:hi] % K], W1[e], W3[e], W2[e])
+        return y
+
+    pin()  # the pin holds for the oracle as it is
+    monkeypatch.setattr(O, "routed_expert_outputs", wrong)
+    with pytest.raises(AssertionError):
+        pin()

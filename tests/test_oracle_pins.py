@@ -367,3 +367,26 @@ def test_select_only_bias_variant():
     i2, g2 = O.topk_gates_select_only_bias(l, b, 3)
     assert np.all(i2[:, 0] == 5)
     np.testing.assert_allclose(g2[:, 0], scipy.special.softmax(l, axis=1)[:, 5], rtol=1e-14)
+
+
+def test_routed_expert_outputs_against_torch():
+    """Every routed slot's row: y[inv[t*K+k]] = FFN_{idx[t,k]}(u_t) (eq. (9)'s
+    routed terms before the gate), against torch's float64 linear / silu
+    evaluated token by token."""
+    rng = np.random.default_rng(11)
+    T, d, I, n, K = 9, 12, 8, 5, 3
+    u = rng.standard_normal((T, d))
+    W1 = rng.standard_normal((n, I, d)) / math.sqrt(d)
+    W3 = rng.standard_normal((n, I, d)) / math.sqrt(d)
+    W2 = rng.standard_normal((n, d, I)) / math.sqrt(I)
+    idx = np.argsort(rng.standard_normal((T, n)), axis=1)[:, :K].astype(np.int32)
+    counts, offsets, perm, inv = O.dispatch(idx, n)
+    y = O.routed_expert_outputs(u, perm, offsets, K, W1, W3, W2)
+    tu = torch.from_numpy(u)
+    for t in range(T):
+        for k in range(K):
+            e = int(idx[t, k])
+            a = F.silu(F.linear(tu[t], torch.from_numpy(W1[e]))) * \
+                F.linear(tu[t], torch.from_numpy(W3[e]))
+            ref = F.linear(a, torch.from_numpy(W2[e])).numpy()
+            np.testing.assert_allclose(y[inv[t * K + k]], ref, rtol=0, atol=1e-12)
