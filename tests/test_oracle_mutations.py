@@ -78,3 +78,33 @@ def test_routed_rows_pin_rejects_a_wrong_token_of_a_slot(monkeypatch):
     monkeypatch.setattr(O, "routed_expert_outputs", wrong)
     with pytest.raises(AssertionError):
         pin()
+
+
+def test_logit_pin_rejects_a_dropped_router_bias(monkeypatch):
+    """Planted mistake: eq. (11)'s logits without the per-expert bias."""
+    from tests.test_oracle_pins import test_router_logits_match_matmul_and_bias as pin
+    orig = O.router_logits
+    pin()
+    monkeypatch.setattr(O, "router_logits", lambda u, E, bias=None, block=None: orig(u, E, None))
+    with pytest.raises(AssertionError):
+        pin()
+
+
+def test_dispatch_pin_rejects_unstable_token_order(monkeypatch):
+    """Planted mistake: each expert's tokens listed in decreasing t."""
+    from tests.test_oracle_pins import test_dispatch_brute_force as pin
+    orig = O.dispatch
+
+    def reversed_segments(idx, n):
+        counts, offsets, perm, inv = orig(idx, n)
+        perm = perm.copy()
+        for e in range(n):
+            perm[offsets[e]:offsets[e + 1]] = perm[offsets[e]:offsets[e + 1]][::-1]
+        inv = np.empty_like(inv)
+        inv[perm] = np.arange(perm.size, dtype=inv.dtype)
+        return counts, offsets, perm, inv
+
+    pin(37, 8, 3)
+    monkeypatch.setattr(O, "dispatch", reversed_segments)
+    with pytest.raises(AssertionError):
+        pin(37, 8, 3)
