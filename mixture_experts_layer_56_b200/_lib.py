@@ -40,6 +40,9 @@ MOE_KERNEL_GEMM_GATE_UP = 4
 MOE_KERNEL_GEMM_DOWN = 5
 MOE_KERNEL_COMBINE = 6
 MOE_KERNEL_FFN_F32 = 7
+MOE_KERNEL_MEMSET = 8
+MOE_KERNEL_PACK = 9
+MOE_KERNEL_BALANCE = 10
 MOE_DISPATCH_STATIC_SCRATCH_BYTES = 512 * 1024
 
 
