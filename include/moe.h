@@ -195,10 +195,14 @@ int moe_layer_forward(const moe_shape_t* shape, const void* u, const void* E,
                       size_t ws_bytes, moe_stream_t stream);
 
 /* moe_layer_forward with the activations in HOST memory: u_host [T, d] is
-   copied to the device, the layer runs, and h is copied back into h_host, all
-   enqueued on `stream`; the call then waits for the stream.  Page-locked
-   host buffers make the copies asynchronous DMA.  Weights stay on the
-   device.  Workspace: moe_workspace_size plus 2*T*d*elem bytes. */
+   copied to the device, the layer runs, and h is copied back into h_host;
+   the call returns when h_host is written.  Page-locked host buffers make
+   the copies asynchronous DMA.  Weights stay on the device.  Batches of at
+   least 4352 tokens run in up to 4 chunks: the uploads and downloads go
+   through two streams of the library's own, overlapping the forward of
+   other chunks on `stream`, and start after the work already on `stream`.
+   h equals moe_layer_forward's bit for bit.  Calls on one device run one
+   at a time.  Workspace: moe_workspace_size plus 2*T*d*elem bytes. */
 int moe_layer_forward_host(const moe_shape_t* shape, const void* u_host,
                            const void* E, const float* bias, const void* W13,
                            const void* W2, const void* W13_s, const void* W2_s,

@@ -372,6 +372,41 @@ bool shared_ptrs_ok(const moe_shape_t& s, const void* W13_s, const void* W2_s) {
   return s.n_shared == 0 || (W13_s && W2_s);
 }
 
+// Chunks of moe_layer_forward_host: each above kMinHostChunk tokens, where the
+// router runs one CTA per 128-token tile with no cluster split, up to 4.
+constexpr int64_t kMinHostChunk = 2176;
+int host_chunks(int64_t T) {
+  const int64_t n = T / kMinHostChunk;
+  return static_cast<int>(n < 1 ? 1 : (n > 4 ? 4 : n));
+}
+
+// Per device: an upload and a download stream and the events that order
+// them against the caller's stream (created once; no device memory).
+struct HostPipe {
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  std::vector<cudaEvent_t> ev;  // [0] start, [1..n] uploads, [n+1..2n] forwards
+  std::mutex busy;              // one host-buffer call at a time per device
+};
+int host_pipe(int nc, HostPipe** out) {
+  static HostPipe pipes[64];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  HostPipe& hp = pipes[dev];
+  if (!hp.s_in &&
+      (cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking) != cudaSuccess ||
+       cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking) != cudaSuccess))
+    return MOE_ERR_CUDA;
+  while (hp.ev.size() < static_cast<size_t>(1 + 2 * nc)) {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return MOE_ERR_CUDA;
+    hp.ev.push_back(e);
+  }
+  *out = &hp;
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -579,17 +614,75 @@ int moe_layer_forward_host(const moe_shape_t* shape, const void* u_host, const v
   DeviceInfo di;
   if (int rc = device_info(&di)) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t bytes = static_cast<size_t>(shape->T) * shape->d * elem_bytes(shape->dtype);
-  void* u_dev = at<void>(ws, L.u_host);
-  void* h_dev = at<void>(ws, L.h_host);
-  if (cudaMemcpyAsync(u_dev, u_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (int rc = forward_device(*shape, L, u_dev, E, bias, W13, W2, W13_s, W2_s, h_dev, ws, st,
-                              di.sms))
+  const size_t row_bytes = static_cast<size_t>(shape->d) * elem_bytes(shape->dtype);
+  const size_t bytes = static_cast<size_t>(shape->T) * row_bytes;
+  uint8_t* u_dev = at<uint8_t>(ws, L.u_host);
+  uint8_t* h_dev = at<uint8_t>(ws, L.h_host);
+  const int nc = host_chunks(shape->T);
+  if (nc == 1) {
+    if (cudaMemcpyAsync(u_dev, u_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (int rc = forward_device(*shape, L, u_dev, E, bias, W13, W2, W13_s, W2_s, h_dev, ws, st,
+                                di.sms))
+      return rc;
+    if (cudaMemcpyAsync(h_host, h_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+  // Chunks of tokens: chunk i's upload and chunk i-1's download overlap the
+  // forward of the chunk between them.  Tokens are independent and every
+  // chunk runs with the whole batch's GEMM tile mode (and above the router's
+  // cluster-split size), so h is the one-pass result bit for bit.
+  HostPipe* hp = nullptr;
+  if (int rc = host_pipe(nc, &hp)) return rc;
+  std::lock_guard<std::mutex> busy(hp->busy);
+  // on an error, nothing may still copy from or to the caller's buffers
+  auto fail = [&](int rc) {
+    cudaStreamSynchronize(hp->s_in);
+    cudaStreamSynchronize(st);
+    cudaStreamSynchronize(hp->s_out);
     return rc;
-  if (cudaMemcpyAsync(h_host, h_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  return cudaStreamSynchronize(st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  };
+  moe_shape_t sc = *shape;
+  if (!(sc.flags & (MOE_FLAG_GEMM_SINGLE_CTA | MOE_FLAG_GEMM_CTA_PAIR))) {
+    const bool pair = shape->T * shape->top_k >= static_cast<int64_t>(shape->n_routed) * 128;
+    sc.flags |= pair ? MOE_FLAG_GEMM_CTA_PAIR : MOE_FLAG_GEMM_SINGLE_CTA;
+  }
+  // the copies start after the caller's earlier work on `stream`
+  if (cudaEventRecord(hp->ev[0], st) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->s_in, hp->ev[0], 0) != cudaSuccess)
+    return fail(MOE_ERR_CUDA);
+  auto chunk = [&](int i, int64_t* t0, int64_t* tn) {
+    *t0 = shape->T * i / nc;
+    *tn = shape->T * (i + 1) / nc - *t0;
+  };
+  for (int i = 0; i < nc; ++i) {
+    int64_t t0, tn;
+    chunk(i, &t0, &tn);
+    if (cudaMemcpyAsync(u_dev + t0 * row_bytes, static_cast<const uint8_t*>(u_host) + t0 * row_bytes,
+                        tn * row_bytes, cudaMemcpyHostToDevice, hp->s_in) != cudaSuccess ||
+        cudaEventRecord(hp->ev[1 + i], hp->s_in) != cudaSuccess)
+      return fail(MOE_ERR_CUDA);
+  }
+  for (int i = 0; i < nc; ++i) {
+    int64_t t0, tn;
+    chunk(i, &t0, &tn);
+    sc.T = tn;
+    const Layout Lc = layout_of(sc);  // intermediates of one chunk (below L's staging)
+    if (cudaStreamWaitEvent(st, hp->ev[1 + i], 0) != cudaSuccess) return fail(MOE_ERR_CUDA);
+    if (int rc = forward_device(sc, Lc, u_dev + t0 * row_bytes, E, bias, W13, W2, W13_s, W2_s,
+                                h_dev + t0 * row_bytes, ws, st, di.sms))
+      return fail(rc);
+    if (cudaEventRecord(hp->ev[1 + nc + i], st) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->s_out, hp->ev[1 + nc + i], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t*>(h_host) + t0 * row_bytes, h_dev + t0 * row_bytes,
+                        tn * row_bytes, cudaMemcpyDeviceToHost, hp->s_out) != cudaSuccess)
+      return fail(MOE_ERR_CUDA);
+  }
+  return cudaStreamSynchronize(hp->s_out) == cudaSuccess &&
+                 cudaStreamSynchronize(st) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 int moe_expert_balance(const moe_shape_t* shape, const void* u, const void* E, const float* bias,

@@ -278,3 +278,22 @@ def test_half_activated_small_shapes():
     wl = W("half_activated", T=1500, d=1280, n_routed=63, n_shared=1, inter=896, top_k=3)
     rep = P.full_parity(S.make_inputs(wl))
     assert rep["gpu"]["counts"].sum() == 1500 * 3
+
+
+def test_host_io_chunked_pipeline_matches_device_path():
+    """Above 4352 tokens the host-buffer call runs in chunks whose copies
+    overlap the forward; h still equals the one-pass device forward bit for
+    bit (same GEMM tile mode for every chunk, no router cluster split)."""
+    for T in (4400, 9000):
+        wl = W(f"hostio{T}", T=T, d=256, n_routed=16, n_shared=1, inter=128, top_k=4)
+        x = S.make_inputs(wl)
+        layer = MoELayer(x, host_io=True)
+        u = to_device(x.u, "cuda:0")
+        ref = to_numpy(layer.forward(u))
+        u_h = u.cpu().pin_memory()
+        h_h = torch.empty_like(u_h).pin_memory()
+        for _ in range(2):
+            h_h.zero_()
+            layer.forward_host(u_h, h_h)
+            assert np.array_equal(to_numpy(h_h), ref)
+        assert layer.status() == 0
