@@ -116,3 +116,14 @@ def test_zero_tokens_is_a_no_op(lib):
 
 def test_launch_counter_starts_at_zero_without_gpu(lib):
     assert L.moe_launch_count() == 0
+
+
+@pytest.mark.parametrize("T", [1, 100, 4400, 9000])
+@pytest.mark.parametrize("dtype", [L.MOE_DTYPE_BF16, L.MOE_DTYPE_F32])
+def test_host_workspace_holds_the_activation_staging(lib, T, dtype):
+    """moe_workspace_size_host = moe_workspace_size + room for u and h
+    (2 T d elements, each region rounded to 256 bytes)."""
+    s = _shape(T=T, dtype=dtype, d=256)
+    el = 2 if dtype == L.MOE_DTYPE_BF16 else 4
+    stage = -(-T * 256 * el // 256) * 256
+    assert L.moe_workspace_size_host(s) == L.moe_workspace_size(s) + 2 * stage
