@@ -127,3 +127,17 @@ def test_host_workspace_holds_the_activation_staging(lib, T, dtype):
     el = 2 if dtype == L.MOE_DTYPE_BF16 else 4
     stage = -(-T * 256 * el // 256) * 256
     assert L.moe_workspace_size_host(s) == L.moe_workspace_size(s) + 2 * stage
+
+
+@pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++11")])
+def test_header_compiles_standalone(lang, std, tmp_path):
+    """include/moe.h is a plain C header: it compiles on its own as C99 and
+    as C++11, with warnings as errors."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    r = subprocess.run([cc, "-x", lang, f"-std={std}", "-Wall", "-Wextra", "-Werror",
+                        "-fsyntax-only", HEADER], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
