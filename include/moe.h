@@ -156,7 +156,10 @@ int moe_dispatch(const moe_shape_t* shape, const int32_t* idx, int32_t* counts,
    larger shapes return MOE_ERR_SCRATCH_LIMIT before any launch.
    Set-up: the first call on each device (current device at the call)
    looks up the array's device address; make that first call before any
-   stream capture begins on the device.
+   stream capture begins on the device.  If that lookup fails the call
+   returns MOE_ERR_CUDA and clears the calling thread's last CUDA error
+   (cudaGetLastError), including an earlier one the caller had not read.
+   Tracing (moe_profile_enable) brackets its kernels as MOE_KERNEL_DISPATCH.
    Sharing: every call in the process, on any stream, uses the same array.
    Calls whose kernels may overlap on a device race on it and corrupt each
    other's perm/inv/offsets; order them (one stream, or events).  Nothing in

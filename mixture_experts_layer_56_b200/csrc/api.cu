@@ -60,32 +60,31 @@ void record_event(cudaEvent_t e, cudaStream_t st) {
     cudaEventRecord(e, st);
 }
 
+}  // namespace
+
 // RAII bracket: records the start event now and the end event when it goes
 // out of scope (after the stage's launches were enqueued).
-class Stage {
- public:
-  Stage(int32_t kind, cudaStream_t st) : st_(st) {
-    Profiler& p = prof();
-    if (!p.on.load() || kind < 0 || kind > 31 || !((p.mask.load() >> kind) & 1u)) return;
-    std::lock_guard<std::mutex> lock(p.mu);
-    if (p.recs.size() >= kMaxProfRecs) return;
-    ProfRec r{kind, p.get(), p.get()};
-    if (!r.beg || !r.end) return;
-    record_event(r.beg, st_);
-    p.recs.push_back(r);
-    idx_ = static_cast<long>(p.recs.size()) - 1;
-  }
-  ~Stage() {
-    if (idx_ < 0) return;
-    Profiler& p = prof();
-    std::lock_guard<std::mutex> lock(p.mu);
-    record_event(p.recs[static_cast<size_t>(idx_)].end, st_);
-  }
+StageScope::StageScope(int32_t kind, cudaStream_t st) : st_(st) {
+  Profiler& p = prof();
+  if (!p.on.load() || kind < 0 || kind > 31 || !((p.mask.load() >> kind) & 1u)) return;
+  std::lock_guard<std::mutex> lock(p.mu);
+  if (p.recs.size() >= kMaxProfRecs) return;
+  ProfRec r{kind, p.get(), p.get()};
+  if (!r.beg || !r.end) return;
+  record_event(r.beg, st_);
+  p.recs.push_back(r);
+  idx_ = static_cast<long>(p.recs.size()) - 1;
+}
 
- private:
-  cudaStream_t st_;
-  long idx_ = -1;
-};
+StageScope::~StageScope() {
+  if (idx_ < 0) return;
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> lock(p.mu);
+  record_event(p.recs[static_cast<size_t>(idx_)].end, st_);
+}
+
+namespace {
+using Stage = StageScope;
 }  // namespace
 
 namespace {

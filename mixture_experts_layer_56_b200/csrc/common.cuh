@@ -91,6 +91,20 @@ __device__ __forceinline__ void pdl_trigger() {
 void count_launch(int n = 1);
 int check_launch();  // MOE_OK or MOE_ERR_CUDA after a <<<>>> launch
 
+// Tracer bracket of one stage (moe_profile_enable): records a start event on
+// `st` when built and an end event when destroyed, if tracing of `kind` is on.
+class StageScope {
+ public:
+  StageScope(int32_t kind, cudaStream_t st);
+  ~StageScope();
+  StageScope(const StageScope&) = delete;
+  StageScope& operator=(const StageScope&) = delete;
+
+ private:
+  cudaStream_t st_;
+  long idx_ = -1;
+};
+
 // A kernel's opt-in dynamic shared-memory size, set on the current device
 // the first time it launches there (the attribute belongs to the device's
 // copy of the kernel; `done` holds one bit per device).

@@ -54,7 +54,9 @@ int scratch_of_current_device(void** out) {
       return MOE_ERR_CUDA;
     if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED;
     if (cudaGetSymbolAddress(&p, g_dispatch_scratch) != cudaSuccess || !p) {
-      cudaGetLastError();  // the failed lookup must not poison later launches
+      // the failed lookup must not surface as a later launch's error; this also
+      // consumes any earlier unread error of the thread (stated in moe.h)
+      cudaGetLastError();
       return MOE_ERR_CUDA;
     }
     g_scratch_addr[dev].store(p, std::memory_order_release);
@@ -86,6 +88,7 @@ int moe_dispatch_static_scratch(const moe_shape_t* shape, const int32_t* idx, in
   if (int rc = scratch_of_current_device(&scratch)) return rc;
   int32_t* chunk_counts = static_cast<int32_t*>(scratch);
   int32_t* chunk_base = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(scratch) + per_array);
+  StageScope sg(MOE_KERNEL_DISPATCH, static_cast<cudaStream_t>(stream));
   return launch_dispatch(idx, shape->T, shape->top_k, shape->n_routed, chunk_counts, chunk_base,
                          counts, offsets, perm, inv, static_cast<cudaStream_t>(stream));
 }

@@ -16,8 +16,19 @@ Bars (the layer's floating-point results are bf16 with fp32 accumulation):
   term is the bf16 output rounding, which alone exceeds 2e-2 once |x| > 5.12)
   and ||x - x_ref||_F / ||x_ref||_F <= 1e-2.
 * fp32 layer: |x - x_ref| <= 1e-4 + 1e-5 |x_ref|, relative Frobenius <= 1e-5.
+
+Every parity run also records the literal figures beside those bars
+(error_stats, gate_stats): the plain max |err| against the fp64 oracle and
+against the oracle rounded to bf16, how many elements exceed 2e-2 (and so
+pass only through the 2^-8 |ref| term) and the largest |ref| among them, the
+relative Frobenius error, and the worst gate error divided by the fp32 model
+2^-24 sqrt(d) L_t s.  With MOE_PARITY_REPORT_DIR set, each report is written
+there as parity_<workload>.json.
 """
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 import torch
@@ -138,6 +149,60 @@ def assert_close(got: np.ndarray, ref: np.ndarray, what: str, bf16: bool = True)
     return float(err.max())
 
 
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """x rounded to float32 and then to bf16 (nearest even), as float64."""
+    return S.bf16_bits_to_f32(S.f32_to_bf16_bits(x.astype(np.float32))).astype(np.float64)
+
+
+def error_stats(got: np.ndarray, ref: np.ndarray, bf16: bool = True) -> dict:
+    """The literal error figures of one output against the fp64 oracle."""
+    err = np.abs(got - ref)
+    atol = 2e-2 if bf16 else 1e-4
+    over = err > atol
+    nref = np.linalg.norm(ref)
+    out = {
+        "elements": int(err.size),
+        "max_abs_err": float(err.max()) if err.size else 0.0,
+        "atol": atol,
+        "n_over_atol": int(over.sum()),
+        "max_abs_ref_where_over_atol": float(np.abs(ref[over]).max()) if over.any() else None,
+        "max_err_minus_atol_over_abs_ref": (float(((err - atol)[over] / np.abs(ref[over])).max())
+                                            if over.any() else None),
+        "rel_fro": float(np.linalg.norm(got - ref) / nref) if nref > 0 else 0.0,
+        "max_abs_ref": float(np.abs(ref).max()) if ref.size else 0.0,
+    }
+    if bf16:
+        out["max_abs_err_vs_bf16_rounded_ref"] = (float(np.abs(got - bf16_round(ref)).max())
+                                                  if err.size else 0.0)
+    return out
+
+
+def gate_stats(w: np.ndarray, idx: np.ndarray, gate_s: np.ndarray, logits: np.ndarray,
+               d: int, mism: np.ndarray) -> dict:
+    """Gate errors (tokens whose selection matches the oracle's) against the
+    fp32 model 2^-24 sqrt(d) L_t s: the ratio the tolerance factor 10 covers."""
+    ok = ~mism
+    g = np.take_along_axis(gate_s, idx.astype(np.int64), axis=1)[ok]
+    err = np.abs(w.astype(np.float64)[ok] - g)
+    L_t = np.abs(logits).max(axis=1, keepdims=True)[ok]
+    model = 2.0 ** -24 * np.sqrt(d) * L_t * g
+    ratio = err / np.maximum(model, 1e-300)
+    return {"max_abs_err": float(err.max()) if err.size else 0.0,
+            "max_rel_err": float((err / np.maximum(g, 1e-300)).max()) if err.size else 0.0,
+            "max_err_over_fp32_model": float(ratio.max()) if err.size else 0.0,
+            "p99_err_over_fp32_model": float(np.quantile(ratio, 0.99)) if err.size else 0.0}
+
+
+def write_report(name: str, rep: dict) -> None:
+    """parity_<name>.json under MOE_PARITY_REPORT_DIR (if set)."""
+    out = os.environ.get("MOE_PARITY_REPORT_DIR")
+    if not out:
+        return
+    os.makedirs(out, exist_ok=True)
+    with open(os.path.join(out, f"parity_{name}.json"), "w") as f:
+        json.dump({k: v for k, v in rep.items() if k != "gpu"}, f, indent=1, sort_keys=True)
+
+
 def full_parity(x: S.LayerInputs, flags: int = 0, device="cuda:0"):
     """Every stage against the oracle, every token.  Returns a report."""
     wl = x.wl
@@ -156,6 +221,8 @@ def full_parity(x: S.LayerInputs, flags: int = 0, device="cuda:0"):
         ref_idx = None
     lb = l if f["bias"] is None else l + f["bias"][None, :]
     near, mism = check_routing(gpu["idx"], gpu["w"], key, wl.top_k, ref_idx, gate_s, lb, wl.d)
+    ref_sel = ref_idx if ref_idx is not None else O.topk_gates(key, wl.top_k)[0]
+    mism_rows = np.any(gpu["idx"] != ref_sel, axis=1)
     check_dispatch(gpu, wl.n_routed)
     # FFN + combine evaluated by the oracle on the GPU's routing
     ref = O.layer_forward(f["u"], f["E"], f["bias"], f["W1"], f["W3"], f["W2"], f["W1_s"],
@@ -166,7 +233,16 @@ def full_parity(x: S.LayerInputs, flags: int = 0, device="cuda:0"):
     esh = assert_close(gpu["ysh"], ref["y_shared"], "ysh", bf16)
     eh = assert_close(gpu["h"], ref_h, "h", bf16)
     assert np.array_equal(gpu["h_raw"], gpu["h_fwd_raw"]), "layer_forward != stage-wise result"
-    return dict(near_ties=near, mismatches=mism, err_y=ey, err_ysh=esh, err_h=eh, gpu=gpu)
+    rep = dict(workload=wl.name, tokens=int(wl.T), tokens_checked=int(wl.T), flags=int(flags),
+               near_ties=near, mismatches=mism, err_y=ey, err_ysh=esh, err_h=eh,
+               h=error_stats(gpu["h"], ref_h, bf16), y=error_stats(gpu["y"], ref["y"], bf16),
+               ysh=error_stats(gpu["ysh"], ref["y_shared"], bf16),
+               gates=gate_stats(gpu["w"], gpu["idx"], gate_s, lb, wl.d, mism_rows),
+               routing="idx/counts/offsets/perm/inv bit-exact on every token (near ties "
+                       "counted)", gpu=gpu)
+    if flags == 0:
+        write_report(wl.name, rep)
+    return rep
 
 
 def sample_tokens(gpu: dict, K: int, n_random: int = 512, seed: int = 0) -> np.ndarray:
@@ -197,6 +273,7 @@ def sampled_parity(x: S.LayerInputs, device="cuda:0", n_random: int = 512):
     l = O.router_logits(f["u"], f["E"], f["bias"])
     s = O.softmax(l)
     near, mism = check_routing(gpu["idx"], gpu["w"], s, wl.top_k, logits=l, d=wl.d)
+    mism_rows = np.any(gpu["idx"] != O.topk_gates(s, wl.top_k)[0], axis=1)
     check_dispatch(gpu, wl.n_routed)
     toks = sample_tokens(gpu, wl.top_k, n_random)
     g = np.take_along_axis(s, gpu["idx"].astype(np.int64), axis=1)
@@ -207,5 +284,14 @@ def sampled_parity(x: S.LayerInputs, device="cuda:0", n_random: int = 512):
     ref_sh = O.shared_experts(f["u"][toks], f["W1_s"], f["W3_s"], f["W2_s"])
     esh = assert_close(gpu["ysh"][toks], ref_sh, "ysh (sampled)")
     assert np.array_equal(gpu["h_raw"], gpu["h_fwd_raw"]), "layer_forward != stage-wise result"
-    return dict(near_ties=near, mismatches=mism, err_h=eh, err_ysh=esh, sampled=int(toks.size),
-                gpu=gpu)
+    rep = dict(workload=wl.name, tokens=int(wl.T), tokens_checked=int(toks.size), flags=0,
+               near_ties=near, mismatches=mism, err_h=eh, err_ysh=esh, sampled=int(toks.size),
+               h=error_stats(gpu["h"][toks], ref_h), ysh=error_stats(gpu["ysh"][toks], ref_sh),
+               gates=gate_stats(gpu["w"], gpu["idx"], s, l, wl.d, mism_rows),
+               routing="idx/counts/offsets/perm/inv bit-exact on every token (near ties "
+                       "counted); h and ysh on the sampled tokens",
+               sample=f"{n_random} random tokens plus every token of the most-loaded expert's "
+                      f"first 128 rows and of each expert's last partial 128-row tile",
+               gpu=gpu)
+    write_report(wl.name, rep)
+    return rep
