@@ -94,6 +94,21 @@ enum {
      up to fp32 summation order.  The fp32 dtype always uses the CUDA
      cores. */
   MOE_FLAG_ROUTER_SIMT = 8,
+  /* Failure injection, for tests of the error path: the TMA producer of each
+     bf16 expert GEMM waits, before its first load, for a shared-memory slot
+     that nothing releases.  That wait gives up after 1 ms like any bounded
+     wait: the kernel records MOE_ERR_DEVICE_CHECK in the workspace status
+     word, lets its in-flight work finish, frees its tensor memory and
+     returns.  The call's outputs are then not valid; the context stays
+     usable.  Never set in production. */
+  MOE_FLAG_INJECT_WAIT_TIMEOUT = 16,
+  /* CTA-pair tiles at most 256 columns wide.  Default (0): where every
+     group's output width is a multiple of 512 (2*inter and 2*inter*n_shared
+     for the gate/up GEMM, d for the down GEMM), a CTA pair computes
+     256 x 512 tiles (two N = 256 MMAs per k-block, 48 rather than 64 bytes
+     of operand tiles per clock of tensor work).  Same results up to fp32
+     summation order inside the tensor cores. */
+  MOE_FLAG_GEMM_NARROW = 32,
 };
 
 /* Layer shape.  Limits: 1 <= n_routed <= 256, 1 <= top_k <= min(n_routed, 32),
@@ -191,7 +206,13 @@ int moe_combine(const moe_shape_t* shape, const void* u, const float* ysh,
                 moe_stream_t stream);
 
 /* The whole layer: route, dispatch, expert FFNs and combine, on `stream`,
-   with every intermediate in `ws`.  Arguments as above; h: [T, d] dtype. */
+   with every intermediate in `ws`.  Arguments as above; h: [T, d] dtype.
+   Decode-sized batches (see moe_forward_path) run as one kernel that
+   streams each activated expert's weights once in units of 64 intermediate
+   rows, with fp32 partial down projections summed in a fixed order; their
+   h matches the oracle within the same bars but is not the stage-wise
+   result bit for bit.  All other batches give exactly the result of
+   moe_route, moe_dispatch, moe_expert_ffn and moe_combine. */
 int moe_layer_forward(const moe_shape_t* shape, const void* u, const void* E,
                       const float* bias, const void* W13, const void* W2,
                       const void* W13_s, const void* W2_s, void* h, void* ws,
@@ -211,6 +232,13 @@ int moe_layer_forward_host(const moe_shape_t* shape, const void* u_host,
                            const void* W2, const void* W13_s, const void* W2_s,
                            void* h_host, void* ws, size_t ws_bytes,
                            moe_stream_t stream);
+
+/* How moe_layer_forward runs `shape`: MOE_PATH_STAGES (router, dispatch,
+   grouped GEMMs, combine) or MOE_PATH_DECODE_LAYER (one kernel for the whole
+   layer: bf16, 1 <= T <= 8, d in {256, 512, 1024, 2048}, inter % 64 == 0,
+   and neither a GEMM tile shape nor failure injection forced in flags). */
+enum { MOE_PATH_STAGES = 0, MOE_PATH_DECODE_LAYER = 1 };
+int moe_forward_path(const moe_shape_t* shape, int32_t* path);
 
 /* Bytes moe_layer_forward_host needs. */
 int moe_workspace_size_host(const moe_shape_t* shape, size_t* bytes);
@@ -250,6 +278,7 @@ enum {
   MOE_KERNEL_MEMSET = 8,
   MOE_KERNEL_PACK = 9,
   MOE_KERNEL_BALANCE = 10,
+  MOE_KERNEL_DECODE_LAYER = 11, /* the whole layer for decode-sized batches */
 };
 int moe_profile_enable(int on);
 int moe_profile_read(int32_t* kinds, float* ms, int32_t max, int32_t* count);

@@ -20,6 +20,8 @@ MOE_FLAG_BIAS_SELECT_ONLY = 1
 MOE_FLAG_GEMM_SINGLE_CTA = 2
 MOE_FLAG_GEMM_CTA_PAIR = 4
 MOE_FLAG_ROUTER_SIMT = 8
+MOE_FLAG_INJECT_WAIT_TIMEOUT = 16
+MOE_FLAG_GEMM_NARROW = 32
 
 MOE_OK = 0
 MOE_ERR_NULLPTR = -1
@@ -43,6 +45,9 @@ MOE_KERNEL_FFN_F32 = 7
 MOE_KERNEL_MEMSET = 8
 MOE_KERNEL_PACK = 9
 MOE_KERNEL_BALANCE = 10
+MOE_KERNEL_DECODE_LAYER = 11
+MOE_PATH_STAGES = 0
+MOE_PATH_DECODE_LAYER = 1
 MOE_DISPATCH_STATIC_SCRATCH_BYTES = 512 * 1024
 
 
@@ -72,6 +77,7 @@ SIGNATURES = {
     "moe_launch_count": (c_uint64, []),
     "moe_workspace_size": (c_int, [_SHAPE, POINTER(c_size_t)]),
     "moe_workspace_size_host": (c_int, [_SHAPE, POINTER(c_size_t)]),
+    "moe_forward_path": (c_int, [_SHAPE, POINTER(c_int32)]),
     "moe_pack_w13": (c_int, [_SHAPE, c_int32, _V, _V, _V, _V]),
     "moe_route": (c_int, [_SHAPE, _V, _V, _V, _V, _V, _V]),
     "moe_dispatch": (c_int, [_SHAPE, _V, _V, _V, _V, _V, _V, c_size_t, _V]),
@@ -158,6 +164,12 @@ def moe_workspace_size_host(shape: MoeShape) -> int:
     _check("moe_workspace_size_host",
            lib().moe_workspace_size_host(ctypes.byref(shape), ctypes.byref(n)))
     return n.value
+
+
+def moe_forward_path(shape: MoeShape) -> int:
+    p = c_int32(0)
+    _check("moe_forward_path", lib().moe_forward_path(ctypes.byref(shape), ctypes.byref(p)))
+    return p.value
 
 
 def moe_pack_w13(shape, n_experts, W1, W3, W13, stream=None):

@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "decode_fused.h"
 #include "gemm_sm100.h"
 #include "kernels.h"
 
@@ -94,7 +95,9 @@ inline size_t round_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
   size_t status, idx, w, counts, offsets, perm, inv, chunk_counts, chunk_base, pstat;
-  size_t xperm, act, act_s, y, ysh, total;
+  size_t xperm, act, act_s, y, ysh;
+  size_t dec_logits, dec_part, dec_sync;  // the decode kernel's (empty unless eligible)
+  size_t total;
   size_t u_host, h_host, total_host;  // extra staging for moe_layer_forward_host
 };
 
@@ -127,6 +130,10 @@ Layout layout_of(const moe_shape_t& s) {
   L.act_s = take(T * ns * I * el);
   L.y = take(T * K * d * el);
   L.ysh = take(T * d * 4);
+  const bool dec = decode_fused_eligible(s);
+  L.dec_logits = take(dec ? T * n * 4 : 0);
+  L.dec_part = take(dec ? decode_partial_rows(s) * d * 4 : 0);
+  L.dec_sync = take(dec ? decode_sync_bytes() : 0);
   L.total = o;
   L.u_host = take(T * d * el);
   L.h_host = take(T * d * el);
@@ -142,7 +149,8 @@ int validate(const moe_shape_t* s) {
       s->inter < 1)
     return MOE_ERR_SHAPE;
   const int32_t known = MOE_FLAG_BIAS_SELECT_ONLY | MOE_FLAG_GEMM_SINGLE_CTA |
-                        MOE_FLAG_GEMM_CTA_PAIR | MOE_FLAG_ROUTER_SIMT;
+                        MOE_FLAG_GEMM_CTA_PAIR | MOE_FLAG_ROUTER_SIMT |
+                        MOE_FLAG_INJECT_WAIT_TIMEOUT | MOE_FLAG_GEMM_NARROW;
   if ((s->flags & ~known) != 0) return MOE_ERR_SHAPE;
   if ((s->flags & MOE_FLAG_GEMM_SINGLE_CTA) && (s->flags & MOE_FLAG_GEMM_CTA_PAIR))
     return MOE_ERR_SHAPE;
@@ -196,13 +204,13 @@ T* at(void* ws, size_t off) {
 int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const int32_t* perm,
                    const int32_t* offsets, const void* W13, const void* W2, const void* W13_s,
                    const void* W2_s, void* y, float* ysh, void* ws, cudaStream_t st, int sms,
-                   bool y_slot_order) {
+                   bool y_slot_order, bool rows_gathered = false) {
   const int64_t T = s.T, K = s.top_k, rows = T * K;
   const int d = s.d, I = s.inter, n = s.n_routed, ns = s.n_shared;
   void* xperm = at<void>(ws, L.xperm);
   void* act = at<void>(ws, L.act);
   void* act_s = at<void>(ws, L.act_s);
-  {
+  if (!rows_gathered) {
     // expert-sorted copies of the routed token rows
     Stage sg(MOE_KERNEL_GATHER, st);
     if (int rc = launch_gather(s.dtype, u, perm, rows, d, static_cast<int>(K), xperm, st))
@@ -257,10 +265,19 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     return bn;
   };
 
+  // CTA pairs take 512-column tiles where both groups' widths allow them
+  const bool narrow = (s.flags & MOE_FLAG_GEMM_NARROW) != 0;
+  auto wide_ok = [&](int64_t n_cols_r, int64_t n_cols_s) {
+    return pair && !narrow && n_cols_r % 512 == 0 && (ns == 0 || n_cols_s % 512 == 0);
+  };
+  auto b_box = [&](int BN) { return static_cast<uint32_t>(BN == 512 ? 128 : (pair ? BN / 2 : BN)); };
+
   // ---- gate/up + SwiGLU ---------------------------------------------------
   {
-    const int BN = pick_bn(2 * I, 2 * I * ns, (2 * I) % 256 == 0 ? 256 : 128, 128);
-    const uint32_t bbox = pair ? BN / 2 : BN;
+    const int BN = wide_ok(2 * I64, 2 * I64 * ns)
+                       ? 512
+                       : pick_bn(2 * I, 2 * I * ns, (2 * I) % 256 == 0 ? 256 : 128, 128);
+    const uint32_t bbox = b_box(BN);
     GemmMaps m;
     bool ok = make_map_bf16(&m.a_r, 2, xperm, d64, rows, 1, d64 * 2, 0, a_rows) &&
               make_map_bf16(&m.b_r, 3, W13, d64, 2 * I64, n, d64 * 2, 2 * I64 * d64 * 2, bbox);
@@ -288,13 +305,16 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     a.ld_s = static_cast<int64_t>(I) * ns;
     a.status = status;
     a.a_rows = static_cast<int32_t>(a_rows);
+    a.inject_wait_timeout = (s.flags & MOE_FLAG_INJECT_WAIT_TIMEOUT) ? 1 : 0;
     Stage sg(MOE_KERNEL_GEMM_GATE_UP, st);
     if (int rc = launch(BN, kEpiSwiGLU, m, a)) return rc;
   }
   // ---- down projection ----------------------------------------------------
   {
-    const int BN = pick_bn(d, d, d % 256 == 0 ? 256 : (d % 128 == 0 ? 128 : 64), 64);
-    const uint32_t bbox = pair ? BN / 2 : BN;
+    const int BN = wide_ok(d64, d64)
+                       ? 512
+                       : pick_bn(d, d, d % 256 == 0 ? 256 : (d % 128 == 0 ? 128 : 64), 64);
+    const uint32_t bbox = b_box(BN);
     GemmMaps m;
     bool ok = make_map_bf16(&m.a_r, 2, act, I64, rows, 1, I64 * 2, 0, a_rows) &&
               make_map_bf16(&m.b_r, 3, W2, I64, d64, n, I64 * 2, d64 * I64 * 2, bbox);
@@ -322,6 +342,7 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     a.ld_s = d;
     a.status = status;
     a.a_rows = static_cast<int32_t>(a_rows);
+    a.inject_wait_timeout = (s.flags & MOE_FLAG_INJECT_WAIT_TIMEOUT) ? 1 : 0;
     Stage sg(MOE_KERNEL_GEMM_DOWN, st);
     if (int rc = launch(BN, kEpiPlain, m, a)) return rc;
   }
@@ -331,6 +352,14 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
 int forward_device(const moe_shape_t& s, const Layout& L, const void* u, const void* E,
                    const float* bias, const void* W13, const void* W2, const void* W13_s,
                    const void* W2_s, void* h, void* ws, cudaStream_t st, int sms) {
+  if (decode_fused_eligible(s)) {
+    // a handful of tokens: the whole layer in one kernel
+    Stage sg(MOE_KERNEL_DECODE_LAYER, st);
+    return launch_decode_fused(s, u, E, bias, W13, W2, W13_s, W2_s, h, at<int32_t>(ws, L.idx),
+                               at<float>(ws, L.w), at<float>(ws, L.dec_logits),
+                               at<float>(ws, L.dec_part), at<void>(ws, L.dec_sync),
+                               at<int32_t>(ws, L.status), sms, st);
+  }
   const int64_t T = s.T;
   const int K = s.top_k, n = s.n_routed;
   int32_t* idx = at<int32_t>(ws, L.idx);
@@ -351,17 +380,20 @@ int forward_device(const moe_shape_t& s, const Layout& L, const void* u, const v
                                T > kDispatchChunk ? chunk_counts : nullptr, &counted))
       return rc;
   }
+  // the dispatch of batches above one chunk also gathers the routed rows
+  const DispatchGather dg{s.dtype, u, s.d, at<void>(ws, L.xperm)};
+  bool gathered = false;
   {
     Stage sg(MOE_KERNEL_DISPATCH, st);
     if (int rc = launch_dispatch(idx, T, K, n, chunk_counts, at<int32_t>(ws, L.chunk_base), counts,
-                                 offsets, perm, inv, st, counted))
+                                 offsets, perm, inv, st, counted, &dg, &gathered))
       return rc;
   }
   // the tensor-core path writes y in token-slot order (the combine then
   // reads each token's rows contiguously); the fp32 path keeps expert order
   const bool slot_order = s.dtype == MOE_DTYPE_BF16;
   if (int rc = run_expert_ffn(s, L, u, perm, offsets, W13, W2, W13_s, W2_s, y, ysh, ws, st, sms,
-                              slot_order))
+                              slot_order, gathered))
     return rc;
   Stage sg(MOE_KERNEL_COMBINE, st);
   return launch_combine(s.dtype, u, ysh, y, w, slot_order ? nullptr : inv, T, s.d, K, h, st);
@@ -477,6 +509,7 @@ const char* moe_kernel_name(int32_t kind) {
     case MOE_KERNEL_MEMSET: return "memset";
     case MOE_KERNEL_PACK: return "pack_w13";
     case MOE_KERNEL_BALANCE: return "expert_balance";
+    case MOE_KERNEL_DECODE_LAYER: return "decode_layer";
     default: return "unknown";
   }
 }
@@ -485,6 +518,13 @@ int moe_workspace_size(const moe_shape_t* shape, size_t* bytes) {
   if (!bytes) return MOE_ERR_NULLPTR;
   if (int rc = validate(shape)) return rc;
   *bytes = layout_of(*shape).total;
+  return MOE_OK;
+}
+
+int moe_forward_path(const moe_shape_t* shape, int32_t* path) {
+  if (!path) return MOE_ERR_NULLPTR;
+  if (int rc = validate(shape)) return rc;
+  *path = decode_fused_eligible(*shape) ? MOE_PATH_DECODE_LAYER : MOE_PATH_STAGES;
   return MOE_OK;
 }
 

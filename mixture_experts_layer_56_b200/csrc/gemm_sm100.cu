@@ -188,6 +188,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
       uint32_t phase = 0;
       uint32_t issued = 0, issued_parity = 0;
       bool ok = true;
+      if (args.inject_wait_timeout) {
+        // slot 0 is released only after a load into it has been consumed,
+        // and none was issued: this wait runs out
+        if (!wait_bounded(empty_bar(0), 0u, abort_p, args.status, kInjectedWaitNs)) ok = false;
+      }
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
         const TileInfo ti = decode_tile(place_tile(tile, total_tiles, workers, n_long), tile_start, G, hs,
                                         args.nt_routed, args.nt_shared);

@@ -32,6 +32,10 @@ struct GroupedGemmArgs {
   // tile's other A rows are left as they are in shared memory and their
   // accumulator rows are never stored.
   int32_t a_rows;
+  // Failure injection (MOE_FLAG_INJECT_WAIT_TIMEOUT): before its first load
+  // the TMA producer waits, with a 1 ms limit, for a shared-memory slot that
+  // nothing releases; the kernel then gives up like on any expired wait.
+  int32_t inject_wait_timeout;
 };
 
 // Tile placement of the persistent GEMMs.  Worker w (a CTA, or a CTA pair)
@@ -69,7 +73,9 @@ int launch_grouped_gemm(int BN, int epi, const GemmMaps& maps, const GroupedGemm
                         int grid, cudaStream_t stream);
 
 // The same GEMM on 2-CTA clusters with 256-row tiles (gemm_sm100_pair.cu).
-// B maps must have box rows BN / 2.  `clusters` CTA pairs are launched.
+// B maps must have box rows BN / 2 (128 for BN = 512, the wide tiles of
+// 256 x 512 whose B rows come in two 128-row boxes per k-block).  `clusters`
+// CTA pairs are launched.
 int launch_grouped_gemm_pair(int BN, int epi, const GemmMaps& maps, const GroupedGemmArgs& args,
                              int clusters, cudaStream_t stream);
 

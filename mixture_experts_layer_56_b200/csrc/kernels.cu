@@ -188,6 +188,99 @@ dispatch_scatter_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n
   }
 }
 
+// Scatter plus gather, for one chunk of kDispatchChunk tokens: the scatter
+// above (warps 0-3, one thread per token), then every warp of the block copies
+// the chunk's token rows of u to their K positions of xperm.  Each row of u is
+// read once and written K times, where a separate gather would read it K
+// times; the expert GEMMs then read xperm as before.
+constexpr int kSgThreads = 512;
+constexpr int kSgCopyUnroll = 8;  // 16-byte vectors a lane holds per row piece
+
+template <int NW, int KMAX, typename TE>
+__global__ void __launch_bounds__(kSgThreads)
+dispatch_scatter_gather_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n,
+                               const int32_t* __restrict__ chunk_base, int32_t* __restrict__ perm,
+                               int32_t* __restrict__ inv, const TE* __restrict__ u, int d,
+                               TE* __restrict__ xperm) {
+  __shared__ int wc[kDispWarps][256];
+  __shared__ int spos[kDispatchChunk][KMAX];
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kDispatchChunk;
+  const bool ranker = warp < kDispWarps;  // warp-uniform
+  const int64_t t = t0 + threadIdx.x;
+  int ek[KMAX];
+  uint32_t mask[NW];
+#pragma unroll
+  for (int w = 0; w < NW; ++w) mask[w] = 0;
+  if (ranker) {
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) ek[k] = (t < T && k < K) ? idx[t * K + k] : -1;
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k)
+#pragma unroll
+      for (int w = 0; w < NW; ++w)
+        if (ek[k] >= 0 && (ek[k] >> 5) == w) mask[w] |= 1u << (ek[k] & 31);
+    warp_counts<NW>(mask, n, warp, lane, wc);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    int run = chunk_base[static_cast<int64_t>(blockIdx.x) * n + e];
+    for (int w = 0; w < kDispWarps; ++w) {
+      const int c = wc[w][e];
+      wc[w][e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  if (ranker) {
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      for (int b = 0; b < 32; ++b) {
+        const int e = w * 32 + b;
+        if (e >= n) break;
+        const bool has = (mask[w] >> b) & 1u;
+        const unsigned bal = __ballot_sync(kFull, has);
+        if (has) {
+          const int pos = wc[warp][e] + __popc(bal & lt);
+          int kk = 0;
+#pragma unroll
+          for (int k = 0; k < KMAX; ++k)
+            if (ek[k] == e) kk = k;
+          const int64_t slot = t * K + kk;
+          perm[pos] = static_cast<int32_t>(slot);
+          inv[slot] = pos;
+          spos[threadIdx.x][kk] = pos;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // copy: warp w takes the chunk's tokens w, w + 16, ...
+  constexpr int V = Vec16<TE>::N;
+  constexpr int U = kSgCopyUnroll;
+  const int nv = d / V;
+  const int64_t rem = T - t0;
+  const int nt = rem < kDispatchChunk ? static_cast<int>(rem) : kDispatchChunk;
+  for (int tl = warp; tl < nt; tl += kSgThreads / 32) {
+    const uint4* src = reinterpret_cast<const uint4*>(u + (t0 + tl) * static_cast<int64_t>(d));
+    for (int c0 = lane; c0 < nv; c0 += 32 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int j = 0; j < U; ++j)
+        if (c0 + 32 * j < nv) v[j] = src[c0 + 32 * j];
+      for (int kk = 0; kk < K; ++kk) {
+        uint4* dst = reinterpret_cast<uint4*>(xperm + static_cast<int64_t>(spos[tl][kk]) * d);
+#pragma unroll
+        for (int j = 0; j < U; ++j)
+          if (c0 + 32 * j < nv) dst[c0 + 32 * j] = v[j];
+      }
+    }
+  }
+}
+
 // The whole dispatch in one block, for batches of at most kDispatchChunk
 // tokens (decode): counts, the scan over experts and the scatter.  Each warp
 // visits only the experts its own tokens chose (a handful at decode sizes).
@@ -555,7 +648,9 @@ inline unsigned grid_for_rows(int64_t rows, int rows_per_block) {
 
 int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_counts,
                     int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* perm,
-                    int32_t* inv, cudaStream_t st, bool counts_ready) {
+                    int32_t* inv, cudaStream_t st, bool counts_ready, const DispatchGather* dg,
+                    bool* gathered) {
+  if (gathered) *gathered = false;
   const int64_t nch = dispatch_num_chunks(T);
   const int nw = (n + 31) / 32;
   if (T == 0) {
@@ -603,6 +698,31 @@ int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_
   if (int r2 = launch_k(dispatch_scan_kernel, 1, 256, 0, st, 1, static_cast<const int32_t*>(chunk_counts),
                         nch, n, chunk_base, counts, offsets))
     return r2;
+  if (dg && dg->xperm) {
+    // scatter and gather in one launch
+    const int bf = dg->dtype == MOE_DTYPE_BF16;
+    rc = MOE_ERR_SHAPE;
+#define MOE_SG_LAUNCH(W, KM, TE)                                                             \
+  launch_k(dispatch_scatter_gather_kernel<W, KM, TE>, grid, kSgThreads, 0, st, 1, idx, T, K, n, \
+           static_cast<const int32_t*>(chunk_base), perm, inv, static_cast<const TE*>(dg->u),   \
+           dg->d, static_cast<TE*>(dg->xperm))
+#define MOE_SG_CASE(W)                                                                       \
+  case W:                                                                                    \
+    rc = bf ? (K <= 8 ? MOE_SG_LAUNCH(W, 8, bf16)                                            \
+                      : K <= 16 ? MOE_SG_LAUNCH(W, 16, bf16) : MOE_SG_LAUNCH(W, 32, bf16))   \
+            : (K <= 8 ? MOE_SG_LAUNCH(W, 8, float)                                           \
+                      : K <= 16 ? MOE_SG_LAUNCH(W, 16, float) : MOE_SG_LAUNCH(W, 32, float)); \
+    break;
+    switch (nw) {
+      MOE_SG_CASE(1) MOE_SG_CASE(2) MOE_SG_CASE(3) MOE_SG_CASE(4)
+      MOE_SG_CASE(5) MOE_SG_CASE(6) MOE_SG_CASE(7) MOE_SG_CASE(8)
+      default: return MOE_ERR_SHAPE;
+    }
+#undef MOE_SG_CASE
+#undef MOE_SG_LAUNCH
+    if (rc == MOE_OK && gathered) *gathered = true;
+    return rc;
+  }
   rc = MOE_ERR_SHAPE;
 #define MOE_SCATTER_CASE(W)                                                                  \
   case W:                                                                                    \

@@ -24,10 +24,22 @@ int launch_router_tc(const void* u, const void* E, const float* bias, int64_t T,
                      int K, int flags, int32_t* idx, float* w, float* pstat, int32_t* status,
                      int32_t* chunk_counts, cudaStream_t st);
 
-// counts_ready: chunk_counts already hold the per-chunk counts of idx
+// Optional gather folded into the dispatch: xperm[p] = u[perm[p] / K].
+struct DispatchGather {
+  int dtype;       // MOE_DTYPE_*
+  const void* u;   // [T, d]
+  int d;
+  void* xperm;     // [T*K, d]
+};
+
+// counts_ready: chunk_counts already hold the per-chunk counts of idx.
+// dg (nullable): batches of more than one dispatch chunk also gather the
+// rows into dg->xperm in the same launch; *gathered (nullable) tells
+// whether that happened (single-chunk batches leave it to launch_gather).
 int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_counts,
                     int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* perm,
-                    int32_t* inv, cudaStream_t st, bool counts_ready = false);
+                    int32_t* inv, cudaStream_t st, bool counts_ready = false,
+                    const DispatchGather* dg = nullptr, bool* gathered = nullptr);
 
 int launch_gather(int dtype, const void* u, const int32_t* perm, int64_t rows, int d, int K,
                   void* xperm, cudaStream_t st);

@@ -53,9 +53,12 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // role of the CTA has given up and raised *abort) it raises *abort, records
 // MOE_ERR_DEVICE_CHECK in the workspace status word and returns false.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s, far above any legitimate wait
+// limit of the wait that MOE_FLAG_INJECT_WAIT_TIMEOUT plants in the GEMMs
+constexpr uint64_t kInjectedWaitNs = 1000000ull;  // 1 ms
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
-                                             int32_t* status) {
+                                             int32_t* status,
+                                             uint64_t timeout_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
@@ -63,7 +66,7 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 255u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      if (global_timer_ns() - t0 > timeout_ns) {
         *abort = 1;
         if (status) *reinterpret_cast<volatile int32_t*>(status) = MOE_ERR_DEVICE_CHECK;
         return false;

@@ -82,7 +82,24 @@ def gpu_stages(x: S.LayerInputs, device="cuda:0", flags=0, layer=None):
     return dict(idx=to_numpy(idx), w=to_numpy(w), counts=to_numpy(counts),
                 offsets=to_numpy(offsets), perm=to_numpy(perm), inv=to_numpy(inv),
                 y=as_f64(y), ysh=as_f64(ysh), h=as_f64(h), h_raw=to_numpy(h),
-                h_fwd_raw=to_numpy(h_fwd), status=status, layer=layer)
+                h_fwd_raw=to_numpy(h_fwd), h_fwd=as_f64(h_fwd), status=status, layer=layer,
+                path=L.moe_forward_path(sh))
+
+
+def check_forward(gpu: dict, ref_h: np.ndarray, near: np.ndarray, bf16: bool, tokens=None):
+    """moe_layer_forward's h: the stage-wise result bit for bit, or (the
+    one-kernel decode path) the oracle within the bars on every token whose
+    K-th and (K+1)-th scores are not a near tie (``near``; its router may
+    choose the other expert there).  Returns the error figures of the
+    forward's h."""
+    h_fwd = gpu["h_fwd"] if tokens is None else gpu["h_fwd"][tokens]
+    if gpu["path"] == L.MOE_PATH_STAGES:
+        assert np.array_equal(gpu["h_raw"], gpu["h_fwd_raw"]), "layer_forward != stage-wise result"
+        return None
+    keep = ~near if tokens is None else ~near[tokens]
+    assert keep.any(), "every token is a near tie: the case checks nothing"
+    assert_close(h_fwd[keep], ref_h[keep], "h (decode layer kernel)", bf16)
+    return error_stats(h_fwd[keep], ref_h[keep], bf16)
 
 
 def near_tie_tokens(s: np.ndarray, K: int) -> np.ndarray:
@@ -180,17 +197,23 @@ def error_stats(got: np.ndarray, ref: np.ndarray, bf16: bool = True) -> dict:
 def gate_stats(w: np.ndarray, idx: np.ndarray, gate_s: np.ndarray, logits: np.ndarray,
                d: int, mism: np.ndarray) -> dict:
     """Gate errors (tokens whose selection matches the oracle's) against the
-    fp32 model 2^-24 sqrt(d) L_t s: the ratio the tolerance factor 10 covers."""
+    bar |w - s| <= 1e-6 + s (1e-5 + F * 2^-24 sqrt(d) L_t), F = 10: the
+    factor each gate needs, (|w - s| - 1e-6 - 1e-5 s) / (2^-24 sqrt(d) L_t s),
+    at worst and at the 99th percentile (0 where the fixed terms cover it),
+    and the same for the gates of at least 1e-3."""
     ok = ~mism
     g = np.take_along_axis(gate_s, idx.astype(np.int64), axis=1)[ok]
     err = np.abs(w.astype(np.float64)[ok] - g)
     L_t = np.abs(logits).max(axis=1, keepdims=True)[ok]
     model = 2.0 ** -24 * np.sqrt(d) * L_t * g
-    ratio = err / np.maximum(model, 1e-300)
+    need = np.maximum(err - 1e-6 - 1e-5 * g, 0.0) / np.maximum(model, 1e-300)
+    big = g >= 1e-3
     return {"max_abs_err": float(err.max()) if err.size else 0.0,
-            "max_rel_err": float((err / np.maximum(g, 1e-300)).max()) if err.size else 0.0,
-            "max_err_over_fp32_model": float(ratio.max()) if err.size else 0.0,
-            "p99_err_over_fp32_model": float(np.quantile(ratio, 0.99)) if err.size else 0.0}
+            "max_rel_err_gates_ge_1e-3": float((err[big] / g[big]).max()) if big.any() else 0.0,
+            "factor_needed_max": float(need.max()) if err.size else 0.0,
+            "factor_needed_p99": float(np.quantile(need, 0.99)) if err.size else 0.0,
+            "factor_needed_max_gates_ge_1e-3": float(need[big].max()) if big.any() else 0.0,
+            "factor_allowed": 10.0}
 
 
 def write_report(name: str, rep: dict) -> None:
@@ -232,8 +255,11 @@ def full_parity(x: S.LayerInputs, flags: int = 0, device="cuda:0"):
     ey = assert_close(gpu["y"], ref["y"], "y", bf16)
     esh = assert_close(gpu["ysh"], ref["y_shared"], "ysh", bf16)
     eh = assert_close(gpu["h"], ref_h, "h", bf16)
-    assert np.array_equal(gpu["h_raw"], gpu["h_fwd_raw"]), "layer_forward != stage-wise result"
+    fwd = check_forward(gpu, ref_h, O.topk_gap(key, wl.top_k) < TIE_GAP, bf16)
     rep = dict(workload=wl.name, tokens=int(wl.T), tokens_checked=int(wl.T), flags=int(flags),
+               forward_path=("decode layer kernel" if gpu["path"] == L.MOE_PATH_DECODE_LAYER
+                             else "stages (bit-equal to the stage-wise calls)"),
+               h_forward=fwd,
                near_ties=near, mismatches=mism, err_y=ey, err_ysh=esh, err_h=eh,
                h=error_stats(gpu["h"], ref_h, bf16), y=error_stats(gpu["y"], ref["y"], bf16),
                ysh=error_stats(gpu["ysh"], ref["y_shared"], bf16),
@@ -283,8 +309,11 @@ def sampled_parity(x: S.LayerInputs, device="cuda:0", n_random: int = 512):
     # shared output on the sample
     ref_sh = O.shared_experts(f["u"][toks], f["W1_s"], f["W3_s"], f["W2_s"])
     esh = assert_close(gpu["ysh"][toks], ref_sh, "ysh (sampled)")
-    assert np.array_equal(gpu["h_raw"], gpu["h_fwd_raw"]), "layer_forward != stage-wise result"
+    fwd = check_forward(gpu, ref_h, O.topk_gap(s, wl.top_k) < TIE_GAP, True, tokens=toks)
     rep = dict(workload=wl.name, tokens=int(wl.T), tokens_checked=int(toks.size), flags=0,
+               forward_path=("decode layer kernel" if gpu["path"] == L.MOE_PATH_DECODE_LAYER
+                             else "stages (bit-equal to the stage-wise calls)"),
+               h_forward=fwd,
                near_ties=near, mismatches=mism, err_h=eh, err_ysh=esh, sampled=int(toks.size),
                h=error_stats(gpu["h"][toks], ref_h), ysh=error_stats(gpu["ysh"][toks], ref_sh),
                gates=gate_stats(gpu["w"], gpu["idx"], s, l, wl.d, mism_rows),

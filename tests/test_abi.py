@@ -66,7 +66,7 @@ def _ws_rc(shape):
     (dict(n_shared=-1), L.MOE_ERR_SHAPE),
     (dict(inter=96), L.MOE_ERR_SHAPE),          # not a multiple of 64
     (dict(d=96), L.MOE_ERR_SHAPE),              # bf16 tensor-core path needs d % 64 == 0
-    (dict(flags=16), L.MOE_ERR_SHAPE),          # unknown flag
+    (dict(flags=64), L.MOE_ERR_SHAPE),          # unknown flag
     (dict(flags=6), L.MOE_ERR_SHAPE),           # both GEMM tile shapes forced
     (dict(T=2**31, top_k=2), L.MOE_ERR_SHAPE),  # T*K positions overflow int32
 ])

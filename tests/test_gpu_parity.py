@@ -31,6 +31,9 @@ CASES = [
       bias_var=0.5),
     W("noshared_bn64", T=517, d=320, n_routed=63, n_shared=0, inter=64, top_k=7),
     W("zipf_router", T=777, d=512, n_routed=40, n_shared=3, inter=128, top_k=5, zipf_s=1.1),
+    # every width a multiple of 512: CTA pairs take 256 x 512 tiles
+    W("wide_tiles", T=1100, d=512, n_routed=12, n_shared=2, inter=256, top_k=3),
+    W("wide_ragged", T=333, d=1024, n_routed=5, n_shared=1, inter=512, top_k=2, bias_var=0.5),
 ]
 
 
@@ -39,7 +42,8 @@ def test_tiny_fp32_config_full():
     print(rep["near_ties"], rep["err_h"])
 
 
-GEMM_MODES = {"single_cta": L.MOE_FLAG_GEMM_SINGLE_CTA, "cta_pair": L.MOE_FLAG_GEMM_CTA_PAIR}
+GEMM_MODES = {"single_cta": L.MOE_FLAG_GEMM_SINGLE_CTA, "cta_pair": L.MOE_FLAG_GEMM_CTA_PAIR,
+              "cta_pair_narrow": L.MOE_FLAG_GEMM_CTA_PAIR | L.MOE_FLAG_GEMM_NARROW}
 
 
 @pytest.mark.parametrize("mode", sorted(GEMM_MODES))
@@ -53,7 +57,7 @@ def test_bf16_cases_full(wl, mode):
 def test_gemm_tile_modes_agree(mode):
     """Both tile shapes give results within the bf16 bar of each other and
     the same routing (the routing does not depend on the GEMM)."""
-    wl = W("modes", T=900, d=256, n_routed=8, n_shared=1, inter=128, top_k=2)
+    wl = W("modes", T=900, d=512, n_routed=8, n_shared=1, inter=256, top_k=2)
     x = S.make_inputs(wl)
     a = P.gpu_stages(x, flags=GEMM_MODES[mode])
     b = P.gpu_stages(x, flags=0)
@@ -297,3 +301,41 @@ def test_host_io_chunked_pipeline_matches_device_path():
             layer.forward_host(u_h, h_h)
             assert np.array_equal(to_numpy(h_h), ref)
         assert layer.status() == 0
+
+
+# Decode-sized batches run the whole layer as one kernel (moe_forward_path):
+# every hidden size it takes, with and without shared experts, a router
+# bias, the selection-only bias, K up to 16 and up to 256 routed experts.
+DECODE_CASES = [
+    W("dec_d256", T=1, d=256, n_routed=16, n_shared=1, inter=128, top_k=4),
+    W("dec_d512_t8", T=8, d=512, n_routed=64, n_shared=2, inter=192, top_k=6, bias_var=0.5),
+    W("dec_d1024_noshared", T=5, d=1024, n_routed=32, n_shared=0, inter=256, top_k=3),
+    W("dec_d2048_k16", T=3, d=2048, n_routed=256, n_shared=1, inter=64, top_k=16, bias_var=4.0),
+    W("dec_d256_t7", T=7, d=256, n_routed=8, n_shared=4, inter=320, top_k=8),
+]
+
+
+@pytest.mark.parametrize("wl", DECODE_CASES, ids=[c.name for c in DECODE_CASES])
+def test_decode_layer_kernel(wl):
+    x = S.make_inputs(wl)
+    layer = MoELayer(x)
+    assert L.moe_forward_path(layer.shape) == L.MOE_PATH_DECODE_LAYER
+    rep = P.full_parity(x)
+    assert rep["h_forward"] is not None
+    print(wl.name, rep["h_forward"])
+
+
+def test_decode_layer_kernel_select_only_bias_and_repeat():
+    wl = W("dec_sel", T=6, d=512, n_routed=24, n_shared=1, inter=128, top_k=4, bias_var=1.0)
+    x = S.make_inputs(wl)
+    rep = P.full_parity(x, flags=L.MOE_FLAG_BIAS_SELECT_ONLY)
+    assert rep["gpu"]["path"] == L.MOE_PATH_DECODE_LAYER
+    # the same call again on the same workspace: bitwise the same h
+    layer = rep["gpu"]["layer"]
+    u = to_device(x.u, "cuda:0")
+    h1 = to_numpy(layer.forward(u))
+    h2 = to_numpy(layer.forward(u))
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    assert np.array_equal(h1, h2)
+    assert np.array_equal(h1, rep["gpu"]["h_fwd_raw"])
