@@ -209,10 +209,11 @@ int moe_combine(const moe_shape_t* shape, const void* u, const float* ysh,
    with every intermediate in `ws`.  Arguments as above; h: [T, d] dtype.
    Decode-sized batches (see moe_forward_path) run as one kernel that
    streams each activated expert's weights once in units of 64 intermediate
-   rows, with fp32 partial down projections summed in a fixed order; their
-   h matches the oracle within the same bars but is not the stage-wise
-   result bit for bit.  All other batches give exactly the result of
-   moe_route, moe_dispatch, moe_expert_ffn and moe_combine. */
+   rows, with fp32 partial down projections summed in a fixed order, and
+   other batches of up to 128 tokens route, dispatch and gather in one
+   kernel; their h matches the oracle within the same bars but is not the
+   stage-wise result bit for bit.  All other batches give exactly the result
+   of moe_route, moe_dispatch, moe_expert_ffn and moe_combine. */
 int moe_layer_forward(const moe_shape_t* shape, const void* u, const void* E,
                       const float* bias, const void* W13, const void* W2,
                       const void* W13_s, const void* W2_s, void* h, void* ws,
@@ -233,11 +234,20 @@ int moe_layer_forward_host(const moe_shape_t* shape, const void* u_host,
                            void* h_host, void* ws, size_t ws_bytes,
                            moe_stream_t stream);
 
-/* How moe_layer_forward runs `shape`: MOE_PATH_STAGES (router, dispatch,
-   grouped GEMMs, combine) or MOE_PATH_DECODE_LAYER (one kernel for the whole
-   layer: bf16, 1 <= T <= 8, d in {256, 512, 1024, 2048}, inter % 64 == 0,
-   and neither a GEMM tile shape nor failure injection forced in flags). */
-enum { MOE_PATH_STAGES = 0, MOE_PATH_DECODE_LAYER = 1 };
+/* How moe_layer_forward runs `shape`:
+   MOE_PATH_DECODE_LAYER: one kernel for the whole layer (bf16, 1 <= T <= 8,
+     d in {256, 512, 1024, 2048}, inter % 64 == 0, and neither a GEMM tile
+     shape nor failure injection forced in flags);
+   MOE_PATH_SMALL_BATCH: router, dispatch and gather in one kernel with fp32
+     CUDA-core logits, then the grouped GEMMs and the combine (other bf16
+     batches of at most 128 tokens with d in {256, 512, 1024, 2048}, without
+     MOE_FLAG_ROUTER_SIMT);
+   MOE_PATH_STAGES: router, dispatch, grouped GEMMs, combine, each as
+     moe_route / moe_dispatch / moe_expert_ffn / moe_combine compute them
+     (h is their result bit for bit).
+   The first two match the oracle within the same bars; their gates follow
+   their own fp32 logits, so h is not the stage-wise result bit for bit. */
+enum { MOE_PATH_STAGES = 0, MOE_PATH_DECODE_LAYER = 1, MOE_PATH_SMALL_BATCH = 2 };
 int moe_forward_path(const moe_shape_t* shape, int32_t* path);
 
 /* Bytes moe_layer_forward_host needs. */

@@ -48,6 +48,7 @@ MOE_KERNEL_BALANCE = 10
 MOE_KERNEL_DECODE_LAYER = 11
 MOE_PATH_STAGES = 0
 MOE_PATH_DECODE_LAYER = 1
+MOE_PATH_SMALL_BATCH = 2
 MOE_DISPATCH_STATIC_SCRATCH_BYTES = 512 * 1024
 
 

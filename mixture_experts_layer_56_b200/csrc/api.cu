@@ -131,9 +131,10 @@ Layout layout_of(const moe_shape_t& s) {
   L.y = take(T * K * d * el);
   L.ysh = take(T * d * 4);
   const bool dec = decode_fused_eligible(s);
-  L.dec_logits = take(dec ? T * n * 4 : 0);
+  const bool front = !dec && decode_front_eligible(s);
+  L.dec_logits = take(dec || front ? T * n * 4 : 0);
   L.dec_part = take(dec ? decode_partial_rows(s) * d * 4 : 0);
-  L.dec_sync = take(dec ? decode_sync_bytes() : 0);
+  L.dec_sync = take(dec || front ? kAlign : 0);
   L.total = o;
   L.u_host = take(T * d * el);
   L.h_host = take(T * d * el);
@@ -278,13 +279,16 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
                        ? 512
                        : pick_bn(2 * I, 2 * I * ns, (2 * I) % 256 == 0 ? 256 : 128, 128);
     const uint32_t bbox = b_box(BN);
+    const int bk = BN == 512 ? kWideBK : 64;  // K per k-block
+    const uint32_t bk32 = static_cast<uint32_t>(bk);
     GemmMaps m;
-    bool ok = make_map_bf16(&m.a_r, 2, xperm, d64, rows, 1, d64 * 2, 0, a_rows) &&
-              make_map_bf16(&m.b_r, 3, W13, d64, 2 * I64, n, d64 * 2, 2 * I64 * d64 * 2, bbox);
+    bool ok = make_map_bf16(&m.a_r, 2, xperm, d64, rows, 1, d64 * 2, 0, a_rows, bk32) &&
+              make_map_bf16(&m.b_r, 3, W13, d64, 2 * I64, n, d64 * 2, 2 * I64 * d64 * 2, bbox,
+                            bk32);
     if (ns > 0) {
-      ok = ok && make_map_bf16(&m.a_s, 2, u, d64, T, 1, d64 * 2, 0, a_rows) &&
+      ok = ok && make_map_bf16(&m.a_s, 2, u, d64, T, 1, d64 * 2, 0, a_rows, bk32) &&
            make_map_bf16(&m.b_s, 3, W13_s, d64, 2 * I64 * ns, 1, d64 * 2, 2 * I64 * ns * d64 * 2,
-                         bbox);
+                         bbox, bk32);
     } else {
       m.a_s = m.a_r;
       m.b_s = m.b_r;
@@ -294,9 +298,9 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     a.offsets = offsets;
     a.n_routed = n;
     a.shared_rows = ns > 0 ? static_cast<int32_t>(T) : 0;
-    a.kb_routed = d / 64;
-    a.kb_shared = d / 64;
-    a.kb_per_expert = d / 64;
+    a.kb_routed = d / bk;
+    a.kb_shared = d / bk;
+    a.kb_per_expert = d / bk;
     a.nt_routed = 2 * I / BN;
     a.nt_shared = 2 * I * ns / BN;
     a.out_r = act;
@@ -315,12 +319,14 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
                        ? 512
                        : pick_bn(d, d, d % 256 == 0 ? 256 : (d % 128 == 0 ? 128 : 64), 64);
     const uint32_t bbox = b_box(BN);
+    const int bk = BN == 512 ? kWideBK : 64;  // K per k-block
+    const uint32_t bk32 = static_cast<uint32_t>(bk);
     GemmMaps m;
-    bool ok = make_map_bf16(&m.a_r, 2, act, I64, rows, 1, I64 * 2, 0, a_rows) &&
-              make_map_bf16(&m.b_r, 3, W2, I64, d64, n, I64 * 2, d64 * I64 * 2, bbox);
+    bool ok = make_map_bf16(&m.a_r, 2, act, I64, rows, 1, I64 * 2, 0, a_rows, bk32) &&
+              make_map_bf16(&m.b_r, 3, W2, I64, d64, n, I64 * 2, d64 * I64 * 2, bbox, bk32);
     if (ns > 0) {
-      ok = ok && make_map_bf16(&m.a_s, 2, act_s, I64 * ns, T, 1, I64 * ns * 2, 0, a_rows) &&
-           make_map_bf16(&m.b_s, 3, W2_s, I64, d64, ns, I64 * 2, d64 * I64 * 2, bbox);
+      ok = ok && make_map_bf16(&m.a_s, 2, act_s, I64 * ns, T, 1, I64 * ns * 2, 0, a_rows, bk32) &&
+           make_map_bf16(&m.b_s, 3, W2_s, I64, d64, ns, I64 * 2, d64 * I64 * 2, bbox, bk32);
     } else {
       m.a_s = m.a_r;
       m.b_s = m.b_r;
@@ -330,9 +336,9 @@ int run_expert_ffn(const moe_shape_t& s, const Layout& L, const void* u, const i
     a.offsets = offsets;
     a.n_routed = n;
     a.shared_rows = ns > 0 ? static_cast<int32_t>(T) : 0;
-    a.kb_routed = I / 64;
-    a.kb_shared = I * ns / 64;
-    a.kb_per_expert = I / 64;
+    a.kb_routed = I / bk;
+    a.kb_shared = I * ns / bk;
+    a.kb_per_expert = I / bk;
     a.nt_routed = d / BN;
     a.nt_shared = d / BN;
     a.out_r = y;
@@ -370,6 +376,23 @@ int forward_device(const moe_shape_t& s, const Layout& L, const void* u, const v
   int32_t* inv = at<int32_t>(ws, L.inv);
   void* y = at<void>(ws, L.y);
   float* ysh = at<float>(ws, L.ysh);
+  if (decode_front_eligible(s)) {
+    // a small batch: router, dispatch and gather in one launch, then the
+    // grouped GEMMs and the combine as below
+    {
+      Stage sg(MOE_KERNEL_ROUTER, st);
+      if (int rc = launch_decode_front(s, u, E, bias, idx, w, at<float>(ws, L.dec_logits), counts,
+                                       offsets, perm, inv, at<void>(ws, L.xperm),
+                                       at<void>(ws, L.dec_sync), at<int32_t>(ws, L.status), sms,
+                                       st))
+        return rc;
+    }
+    if (int rc = run_expert_ffn(s, L, u, perm, offsets, W13, W2, W13_s, W2_s, y, ysh, ws, st, sms,
+                                /*y_slot_order=*/true, /*rows_gathered=*/true))
+      return rc;
+    Stage sg(MOE_KERNEL_COMBINE, st);
+    return launch_combine(s.dtype, u, ysh, y, w, nullptr, T, s.d, K, h, st);
+  }
   // batches of more than one dispatch chunk: the router also counts
   int32_t* chunk_counts = at<int32_t>(ws, L.chunk_counts);
   bool counted = false;
@@ -524,7 +547,9 @@ int moe_workspace_size(const moe_shape_t* shape, size_t* bytes) {
 int moe_forward_path(const moe_shape_t* shape, int32_t* path) {
   if (!path) return MOE_ERR_NULLPTR;
   if (int rc = validate(shape)) return rc;
-  *path = decode_fused_eligible(*shape) ? MOE_PATH_DECODE_LAYER : MOE_PATH_STAGES;
+  *path = decode_fused_eligible(*shape)   ? MOE_PATH_DECODE_LAYER
+          : decode_front_eligible(*shape) ? MOE_PATH_SMALL_BATCH
+                                          : MOE_PATH_STAGES;
   return MOE_OK;
 }
 

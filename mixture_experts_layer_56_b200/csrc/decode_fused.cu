@@ -4,33 +4,41 @@
 // At a handful of tokens the layer is a stream of the activated experts'
 // weights (W1/W3/W2 of every routed expert some token chose, plus the shared
 // experts, all read once), so what matters is that every SM streams weights
-// all the time.  The work is cut into units: one unit is kDecUC intermediate
-// rows of one expert (a 128-row packed W13 block [gate 64 | up 64] and the
-// matching 64 columns of W2), for the tokens that chose that expert (all
-// tokens for a shared expert).  A unit computes a = SiLU(W1 x) * (W3 x) for
-// its 64 rows and its partial down projection W2[:, chunk] a, an fp32 row of
-// d values per token, written to its own slot of the workspace.  CTAs take
-// units from an atomic counter, so the units spread evenly whatever the
-// routing; the partial slots are fixed by the unit and the sums below run in
-// a fixed order, so the result is the same whichever CTA took which unit.
+// all the time.  The work is cut into units: one unit is kDecUC = 64
+// intermediate rows of one expert, i.e. one 128-row packed W13 block
+// [gate 64 | up 64] and the matching 64 columns of W2.  CTAs take units from
+// an atomic counter, so the units spread evenly over the SMs whatever the
+// routing; each unit writes fp32 partial down projections into slots fixed by
+// the unit, and the sums below run in a fixed order, so the result does not
+// depend on which CTA took which unit.
 //
-// Phases, all in this one launch (one CTA per SM, 8 compute warps plus a
-// producer warp):
+// A unit on the tensor cores (weights as the M = 128 operand, the batch's
+// tokens as N = 16 columns, fp32 accumulators in TMEM):
+//   gate/up  D1[128 x 16] = W13 block [128 x d] . U^T, U = all tokens (bf16,
+//            zero rows past T), in d/64 MMA steps from TMA tiles;
+//   SwiGLU   a[r, t] = SiLU(D1[r, t]) * D1[64 + r, t]   (r < 64), bf16;
+//   down     D2[m][128 x 16] = W2[m*128 .. +127, chunk cols] . a, d/128 tiles;
+//   store    the columns of the unit's own tokens (its expert's tokens, or all
+//            of them for a shared expert) as partial rows.
+// Roles (8 warps): warp 0 the TMA producer (unit counter, W13 and W2 tiles into
+// an 8-stage ring, running ahead into the next unit), warp 1 the MMA issuer,
+// warp 2 the TMEM owner, warps 4-7 the epilogue (TMEM lane quarters).
+//
+// Phases, all in this one launch (one CTA per SM):
 //  1. Router (CTAs 0 .. ceil(n/8)-1): logits u_t . e_i for 8 experts each,
-//     all tokens, fp32 FMA chains; the CTA that finishes last runs softmax
-//     and top-K for every token (lower expert index first on ties, gates not
-//     renormalised) and publishes idx / w.
+//     all tokens, fp32 FMA chains per lane plus a fixed shuffle tree; the CTA
+//     that finishes last runs softmax and top-K for every token (lower expert
+//     index first on ties, gates not renormalised) and publishes idx / w.
 //  2. Units: the shared experts' units need no routing and come first; the
 //     routed units (active experts in increasing index, chunks in order)
-//     become known once the routing is published.  The producer warp takes
-//     units, streams each unit's W13 block with bulk copies and its W2
-//     columns with TMA into a 4-stage ring, running ahead into the next
-//     unit; the compute warps take the units from a small queue.
-//  3. Combine: once every unit is done, h_t = u_t + sum over the shared
-//     partials + sum_k w[t,k] * (sum over expert idx[t,k]'s partials), in
-//     fp32 in that order, rounded once to bf16.
+//     become known once the routing is published.
+//  3. Combine: once every unit is done, h_t = u_t + sum_j g_j p_j over the
+//     token's partial rows p_j (the shared units' with g = 1, then each
+//     routed slot k's chunks with g = w[t,k]), in fp32: one warp per (token,
+//     4 columns), lane l summing rows l, l + 32, ... in order, then a fixed
+//     shuffle tree; u is added last and h rounded once to bf16.
 // Every wait is bounded: a wait that runs out records MOE_ERR_DEVICE_CHECK in
-// the status word and the kernel winds down without touching h.
+// the status word and the kernel winds down without writing h.
 #include <cuda.h>
 #include <math_constants.h>
 
@@ -45,17 +53,18 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kDecWarps = 8;                         // compute warps
-constexpr int kDecThreads = (kDecWarps + 1) * 32;    // + the producer warp
+constexpr int kDecThreads = 256;                     // 8 warps
 constexpr int kDecUC = 64;                           // intermediate rows per unit
-constexpr int kDecStageBytes = 32 * 1024;
-constexpr int kDecStages = 4;
+constexpr int kDecN = 16;                            // token columns of an MMA
+constexpr int kDecTileBytes = 128 * 64 * 2;          // one 128 x 64 bf16 TMA tile
+constexpr int kDecStages = 8;
 constexpr int kDecQueue = 4;                         // unit descriptors in flight
-constexpr int kDecW2Rows = 256;                      // W2 rows per TMA box
 constexpr int kDecRouterExperts = 8;                 // experts per router CTA
 constexpr int kDecMaxSlots = kDecMaxT * 32;          // routed (token, k) slots
+constexpr uint32_t kDecTmemCols = 512;               // D1 (16) + D2 (16 per 128 rows of d)
+static_assert(kDecMaxT <= kDecN, "the batch fits one MMA's columns");
 
-// sync words at the start of the decode scratch (zeroed before each launch)
+// sync words of the decode scratch (zeroed before each launch)
 struct DecSync {
   int unit_next;     // next unit to take
   int route_arrive;  // router CTAs done with their logits
@@ -67,8 +76,6 @@ struct DecArgs {
   const bf16* u;        // [T, d]
   const bf16* E;        // [n, d]
   const float* bias;    // [n] or null
-  const bf16* W13;      // [n, 2I, d] packed
-  const bf16* W13_s;    // [Ks, 2I, d] packed (null when Ks = 0)
   bf16* h;              // [T, d]
   int32_t* idx;         // [T, K] (workspace)
   float* w;             // [T, K] (workspace)
@@ -79,40 +86,30 @@ struct DecArgs {
   int T, d, n, Ks, I, K, flags;
 };
 
-struct UnitDesc {
+struct __align__(16) UnitDesc {
   int kind;      // 0 shared, 1 routed, -1 no more units
   int expert;    // routed expert e, or shared expert s
   int chunk;     // which kDecUC rows of I
-  int n_tok;
-  int tok_off;   // into the token list (routed) or -1 (all tokens)
   int slot;      // first partial row
+  int8_t row_of[kDecN];  // token t -> its row within the unit's slots, or -1
 };
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-      : "memory");
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 epilogue warps
 }
 
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32) : "memory");
-}
-
-// All compute warps vote: true when every one of them passes true.  Every
-// compute warp reaches each vote exactly once, whatever its own wait saw, so
-// they stay in step also when a wait runs out.
-__device__ __forceinline__ bool consumer_all(bool v) {
+// The 4 epilogue warps vote: true when all of them pass true.  Each of them
+// reaches every vote once, whatever its own wait saw, so they leave the unit
+// loop together also when a wait runs out.
+__device__ __forceinline__ bool epi_all(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 1, %2, q;\n\t"
+      "bar.red.and.pred p, 1, 128, q;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "n"(kDecWarps * 32)
+      : "r"(static_cast<uint32_t>(v))
       : "memory");
   return r != 0;
 }
@@ -142,97 +139,123 @@ __device__ __forceinline__ bool spin_until(const int* p, int target, int32_t* st
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
+// byte offset of element (row, k) in a K-major [rows x 64] bf16 tile with
+// 128-byte swizzle (16-byte chunk k/8 of a row sits at chunk (k/8) ^ (row % 8))
+__device__ __forceinline__ uint32_t sw128_off(int row, int k) {
+  return static_cast<uint32_t>(row * 128 + ((((k >> 3) ^ (row & 7)) & 7) << 4) + (k & 7) * 2);
+}
+
 template <int NV>
 __global__ void __launch_bounds__(kDecThreads, 1)
-decode_layer_kernel(const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmW2s,
-                    const DecArgs a) {
-  constexpr int D = NV * 256;  // hidden size: NV 16-byte chunks per lane
+decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
+                    const __grid_constant__ CUtensorMap tmW13s,
+                    const __grid_constant__ CUtensorMap tmW2,
+                    const __grid_constant__ CUtensorMap tmW2s, const DecArgs a) {
+  constexpr int D = NV * 256;        // hidden size
+  constexpr int KB13 = D / 64;       // gate/up k-blocks per unit
+  constexpr int MT2 = D / 128;       // down row tiles per unit
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, kDecN);
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[2 * kDecStages + 2 * kDecQueue];
+  __shared__ __align__(8) uint64_t bars[2 * kDecStages + 2 * kDecQueue + 4];
   __shared__ UnitDesc qdesc[kDecQueue];
+  __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
-  __shared__ int s_cnt[256], s_off[257], s_active[256], s_nactive;
+  __shared__ int s_cnt[256], s_off[257], s_active[256];
   __shared__ int s_tok[kDecMaxSlots];             // tokens of each expert, increasing t
   __shared__ int s_rank[kDecMaxSlots];            // rank of token t within expert idx[t,k]
   __shared__ int s_idx[kDecMaxSlots];
-  __shared__ int s_total, s_tables_ok, s_last;
-  __shared__ float zbuf[128][kDecMaxT];
-  __shared__ float abuf[kDecUC][kDecMaxT];
+  __shared__ int s_total, s_last;
+  __shared__ float upx[64][kDecN + 1];            // the up rows of D1, for the SwiGLU
 
+  // dynamic: ring | U (KB13 tiles of 16 rows) | a^T (one 16-row tile)
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  float* uf = reinterpret_cast<float*>(ring + kDecStages * kDecStageBytes);  // [T][D] fp32
+  uint8_t* ut = ring + kDecStages * kDecTileBytes;
+  uint8_t* at = ut + KB13 * (kDecN * 128);
   const uint32_t ring_base = smem_addr(ring);
+  const uint32_t ut_base = smem_addr(ut);
+  const uint32_t at_base = smem_addr(at);
   const uint32_t bar_base = smem_addr(bars);
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (kDecStages + s); };
   auto qfull_bar = [&](int q) { return bar_base + 8u * (2 * kDecStages + q); };
   auto qempty_bar = [&](int q) { return bar_base + 8u * (2 * kDecStages + kDecQueue + q); };
+  const uint32_t gu_full = bar_base + 8u * (2 * kDecStages + 2 * kDecQueue);
+  const uint32_t a_ready = gu_full + 8u;
+  const uint32_t dn_full = gu_full + 16u;
+  const uint32_t drain_bar = gu_full + 24u;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = a.T, n = a.n, K = a.K, I = a.I, Ks = a.Ks;
   const int nc = I / kDecUC;
   const int S = Ks * nc;                      // shared units
-  const int rs = 16384 / D;                   // W13 rows per 32 KB stage
-  const int n13 = 128 / rs;                   // W13 stages per unit
-  const int n2 = (D + kDecW2Rows - 1) / kDecW2Rows;  // W2 boxes per unit
   volatile int* abort_p = &abort_flag;
 
   if (tid == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), kDecWarps);
+      mbar_init(empty_bar(s), 1);
     }
     for (int q = 0; q < kDecQueue; ++q) {
       mbar_init(qfull_bar(q), 1);
-      mbar_init(qempty_bar(q), kDecWarps);
+      mbar_init(qempty_bar(q), 5);  // the MMA thread and the 4 epilogue warps
     }
+    mbar_init(gu_full, 1);
+    mbar_init(a_ready, 1);
+    mbar_init(dn_full, 1);
+    mbar_init(drain_bar, 1);
     abort_flag = 0;
-    s_tables_ok = 0;
     fence_mbar_init();
-    fence_async_shared();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_addr(&tmem_slot), kDecTmemCols);
+    tmem_relinquish();
   }
   pdl_wait();  // u, the weights and the zeroed sync words come from earlier stream work
   pdl_trigger();
-  // the batch's token rows, widened to fp32 once
-  for (int i = tid; i < T * (D / 8); i += kDecThreads) {
+  // U: every token row as K-major 64-column tiles with 128-byte swizzle,
+  // zero rows past T (the B operand of every gate/up MMA)
+  for (int i = tid; i < kDecN * (D / 8); i += kDecThreads) {
     const int t = i / (D / 8), c = i - t * (D / 8);
-    const uint4 v = reinterpret_cast<const uint4*>(a.u + static_cast<int64_t>(t) * D)[c];
-    float* dst = uf + t * D + c * 8;
-    reinterpret_cast<float4*>(dst)[0] = make_float4(bf_lo(v.x), bf_hi(v.x), bf_lo(v.y), bf_hi(v.y));
-    reinterpret_cast<float4*>(dst)[1] = make_float4(bf_lo(v.z), bf_hi(v.z), bf_lo(v.w), bf_hi(v.w));
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (t < T) v = reinterpret_cast<const uint4*>(a.u + static_cast<int64_t>(t) * D)[c];
+    *reinterpret_cast<uint4*>(ut + (c >> 3) * (kDecN * 128) + sw128_off(t, (c & 7) * 8)) = v;
   }
+  fence_async_shared();  // generic-proxy writes of U, before the tensor cores read them
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
 
   // ---- 1. router -----------------------------------------------------------
   const int n_rctas = (n + kDecRouterExperts - 1) / kDecRouterExperts;
   if (static_cast<int>(blockIdx.x) < n_rctas) {
-    if (warp < kDecWarps) {
-      const int e = blockIdx.x * kDecRouterExperts + warp;
-      if (e < n) {
-        const uint4* er = reinterpret_cast<const uint4*>(a.E + static_cast<int64_t>(e) * D);
-        float ev[NV][8];
+    const int e = blockIdx.x * kDecRouterExperts + warp;
+    if (e < n) {
+      const uint4* er = reinterpret_cast<const uint4*>(a.E + static_cast<int64_t>(e) * D);
+      float ev[NV][8];
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const uint4 x = er[v * 32 + lane];
+        ev[v][0] = bf_lo(x.x); ev[v][1] = bf_hi(x.x); ev[v][2] = bf_lo(x.y); ev[v][3] = bf_hi(x.y);
+        ev[v][4] = bf_lo(x.z); ev[v][5] = bf_hi(x.z); ev[v][6] = bf_lo(x.w); ev[v][7] = bf_hi(x.w);
+      }
+      for (int t = 0; t < T; ++t) {
+        const uint4* ur = reinterpret_cast<const uint4*>(a.u + static_cast<int64_t>(t) * D);
+        uint4 uv[NV];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) uv[v] = ur[v * 32 + lane];
+        float acc = 0.0f;
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
-          const uint4 x = er[v * 32 + lane];
-          ev[v][0] = bf_lo(x.x); ev[v][1] = bf_hi(x.x); ev[v][2] = bf_lo(x.y); ev[v][3] = bf_hi(x.y);
-          ev[v][4] = bf_lo(x.z); ev[v][5] = bf_hi(x.z); ev[v][6] = bf_lo(x.w); ev[v][7] = bf_hi(x.w);
+          acc = fmaf(bf_lo(uv[v].x), ev[v][0], acc); acc = fmaf(bf_hi(uv[v].x), ev[v][1], acc);
+          acc = fmaf(bf_lo(uv[v].y), ev[v][2], acc); acc = fmaf(bf_hi(uv[v].y), ev[v][3], acc);
+          acc = fmaf(bf_lo(uv[v].z), ev[v][4], acc); acc = fmaf(bf_hi(uv[v].z), ev[v][5], acc);
+          acc = fmaf(bf_lo(uv[v].w), ev[v][6], acc); acc = fmaf(bf_hi(uv[v].w), ev[v][7], acc);
         }
-        for (int t = 0; t < T; ++t) {
-          float acc = 0.0f;
 #pragma unroll
-          for (int v = 0; v < NV; ++v) {
-            const float4* up = reinterpret_cast<const float4*>(uf + t * D + (v * 32 + lane) * 8);
-            const float4 p0 = up[0], p1 = up[1];
-            acc = fmaf(p0.x, ev[v][0], acc); acc = fmaf(p0.y, ev[v][1], acc);
-            acc = fmaf(p0.z, ev[v][2], acc); acc = fmaf(p0.w, ev[v][3], acc);
-            acc = fmaf(p1.x, ev[v][4], acc); acc = fmaf(p1.y, ev[v][5], acc);
-            acc = fmaf(p1.z, ev[v][6], acc); acc = fmaf(p1.w, ev[v][7], acc);
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-          if (lane == 0) a.logits[t * n + e] = acc;
-        }
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) a.logits[t * n + e] = acc;
       }
     }
     __threadfence();
@@ -243,17 +266,16 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW2, const __grid_const
       // the last router CTA: softmax and top-K of every token, warp per token
       __threadfence();
       const bool select_only = (a.flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
-      for (int t = warp; t < T && warp < kDecWarps; t += kDecWarps) {
+      for (int t = warp; t < T; t += kDecThreads / 32) {
         float lg[8], key[8], ex[8];
         float m = -CUDART_INF_F;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const int e = lane + 32 * q;
+          const int ee = lane + 32 * q;
           float l = -CUDART_INF_F, kv = -CUDART_INF_F;
-          if (e < n) {
-            const float raw = __ldcg(a.logits + t * n + e);
-            const float b = a.bias ? a.bias[e] : 0.0f;
-            kv = raw + b;
+          if (ee < n) {
+            const float raw = __ldcg(a.logits + t * n + ee);
+            kv = raw + (a.bias ? a.bias[ee] : 0.0f);
             l = select_only ? raw : kv;
           }
           lg[q] = l;
@@ -277,10 +299,10 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW2, const __grid_const
           int bi = 0x7fffffff;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const int e = lane + 32 * q;
-            if (!((taken >> q) & 1u) && e < n && (key[q] > bv || bi == 0x7fffffff)) {
+            const int ee = lane + 32 * q;
+            if (!((taken >> q) & 1u) && ee < n && (key[q] > bv || bi == 0x7fffffff)) {
               bv = key[q];
-              bi = e;
+              bi = ee;
             }
           }
 #pragma unroll
@@ -313,11 +335,15 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW2, const __grid_const
   }
 
   // ---- 2. units --------------------------------------------------------------
-  if (warp == kDecWarps) {
-    // ------------------------------------------------------- producer warp ----
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer ----
     if (lane == 0) {
+      tma_prefetch_desc(&tmW13);
       tma_prefetch_desc(&tmW2);
-      if (Ks > 0) tma_prefetch_desc(&tmW2s);
+      if (Ks > 0) {
+        tma_prefetch_desc(&tmW13s);
+        tma_prefetch_desc(&tmW2s);
+      }
       int q = 0, stage = 0;
       uint32_t qphase = 0, sphase = 0;
       bool have_tables = false, ok = true;
@@ -326,7 +352,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW2, const __grid_const
         const int u = atomicAdd(&a.sync->unit_next, 1);
         if (u >= S && !have_tables) {
           // the routed units need the routing: build the expert tables
-          if (!spin_until(&a.sync->route_done, 1, a.status)) { *abort_p = 1; ok = false; break; }
+          if (!spin_until(&a.sync->route_done, 1, a.status)) { ok = false; break; }
           for (int e = 0; e < n; ++e) s_cnt[e] = 0;
           for (int i = 0; i < T * K; ++i) {
             const int e = __ldcg(a.idx + i);
@@ -341,60 +367,56 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW2, const __grid_const
           }
           s_off[n] = run;
           for (int i = 0; i < T * K; ++i) s_tok[s_off[s_idx[i]] + s_rank[i]] = i / K;
-          s_nactive = na;
           s_total = S + na * nc;
-          s_tables_ok = 1;
           have_tables = true;
         }
         UnitDesc ud;
+        for (int t = 0; t < kDecN; ++t) ud.row_of[t] = -1;
         if (have_tables && u >= s_total) {
           ud.kind = -1;
+          ud.expert = ud.chunk = ud.slot = 0;
         } else if (u < S) {
           ud.kind = 0;
           ud.expert = u / nc;
           ud.chunk = u - ud.expert * nc;
-          ud.n_tok = T;
-          ud.tok_off = -1;
           ud.slot = u * T;
+          for (int t = 0; t < T; ++t) ud.row_of[t] = static_cast<int8_t>(t);
         } else {
           const int j = (u - S) / nc;
           const int e = s_active[j];
           ud.kind = 1;
           ud.expert = e;
           ud.chunk = (u - S) - j * nc;
-          ud.n_tok = s_cnt[e];
-          ud.tok_off = s_off[e];
           ud.slot = S * T + s_off[e] * nc + ud.chunk * s_cnt[e];
+          for (int r = 0; r < s_cnt[e]; ++r)
+            ud.row_of[s_tok[s_off[e] + r]] = static_cast<int8_t>(r);
         }
         if (!wait_bounded(qempty_bar(q), qphase ^ 1u, abort_p, a.status)) { ok = false; break; }
         qdesc[q] = ud;
         mbar_arrive(qfull_bar(q));  // release: the descriptor and the tables
         if (++q == kDecQueue) { q = 0; qphase ^= 1u; }
         if (ud.kind < 0) break;
-        // the unit's weights: its W13 block in n13 bulk copies, then W2's
-        // columns chunk*64 .. +63 in n2 boxes of 256 rows
-        const bf16* w13 = ud.kind == 0
-                              ? a.W13_s + (static_cast<int64_t>(ud.expert) * 2 * I + ud.chunk * 128) * D
-                              : a.W13 + (static_cast<int64_t>(ud.expert) * 2 * I + ud.chunk * 128) * D;
-        for (int st = 0; st < n13 + n2 && ok; ++st) {
+        // the unit's weights: its W13 block in KB13 tiles of 64 columns of d,
+        // then W2's rows in MT2 tiles of 128, columns chunk*64 .. +63
+        const CUtensorMap* m13 = ud.kind == 0 ? &tmW13s : &tmW13;
+        const CUtensorMap* m2 = ud.kind == 0 ? &tmW2s : &tmW2;
+        const int row13 = ud.expert * 2 * I + ud.chunk * 128;
+        for (int st = 0; st < KB13 + MT2 && ok; ++st) {
           if (!wait_bounded(empty_bar(stage), sphase ^ 1u, abort_p, a.status)) { ok = false; break; }
-          const uint32_t dst = ring_base + stage * kDecStageBytes;
-          if (st < n13) {
-            mbar_arrive_expect_tx(full_bar(stage), kDecStageBytes);
-            bulk_load(dst, w13 + static_cast<int64_t>(st) * rs * D, kDecStageBytes, full_bar(stage));
-          } else {
-            const int box = st - n13;
-            mbar_arrive_expect_tx(full_bar(stage), kDecW2Rows * 128);
-            tma_load_2d(dst, ud.kind == 0 ? &tmW2s : &tmW2, full_bar(stage), ud.chunk * kDecUC,
-                        ud.expert * D + box * kDecW2Rows);
-          }
+          const uint32_t dst = ring_base + stage * kDecTileBytes;
+          mbar_arrive_expect_tx(full_bar(stage), kDecTileBytes);
+          if (st < KB13)
+            tma_load_2d(dst, m13, full_bar(stage), st * 64, row13);
+          else
+            tma_load_2d(dst, m2, full_bar(stage), ud.chunk * kDecUC,
+                        ud.expert * D + (st - KB13) * 128);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (sphase << stage);
           if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
         }
       }
       if (!ok) {
-        // a wait ran out: tell the compute warps, and let the copies in flight land
+        // a wait ran out: the others see the flag; let the loads in flight land
         *abort_p = 1;
         for (int s = 0; s < kDecStages; ++s)
           if (issued & (1u << s)) {
@@ -404,97 +426,126 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW2, const __grid_const
       }
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------- compute warps ----
-    int q = 0, stage = 0;
-    uint32_t qphase = 0, sphase = 0;
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer ----
+    if (lane == 0) {
+      int q = 0, stage = 0;
+      uint32_t qphase = 0, sphase = 0;
+      uint32_t j = 0;
+      bool ok = true;
+      while (ok) {
+        if (!wait_bounded(qfull_bar(q), qphase, abort_p, a.status)) { ok = false; break; }
+        const int kind = qdesc[q].kind;
+        mbar_arrive(qempty_bar(q));
+        if (++q == kDecQueue) { q = 0; qphase ^= 1u; }
+        if (kind < 0) break;
+        // gate/up: D1 = W13 block . U^T
+        for (int kb = 0; kb < KB13; ++kb) {
+          if (!wait_bounded(full_bar(stage), sphase, abort_p, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = ring_base + stage * kDecTileBytes;
+          const uint32_t sb = ut_base + kb * (kDecN * 128);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16(tmem_base, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32),
+                     IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+          mma_commit(empty_bar(stage));
+          if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(gu_full);
+        // down, once the epilogue has read D1 and written a^T
+        if (!wait_bounded(a_ready, j & 1u, abort_p, a.status)) { ok = false; break; }
+        tc_fence_after();
+        for (int m = 0; m < MT2; ++m) {
+          if (!wait_bounded(full_bar(stage), sphase, abort_p, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = ring_base + stage * kDecTileBytes;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16(tmem_base + kDecN + m * kDecN, desc_kmajor_sw128(sa + k * 32),
+                     desc_kmajor_sw128(at_base + k * 32), IDESC, k > 0 ? 1u : 0u);
+          mma_commit(empty_bar(stage));
+          if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(dn_full);
+        ++j;
+      }
+      if (!ok) {
+        *abort_p = 1;
+        // wait for every MMA already issued before TMEM is released
+        mma_commit(drain_bar);
+        int dummy = 0;
+        wait_bounded(drain_bar, 0, &dummy, nullptr);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ----------------------------------------------------------- epilogue ----
+    const int q4 = warp - 4;            // TMEM lane quarter
+    const int r = q4 * 32 + lane;       // TMEM lane: W13 block row / W2 row in a tile
+    const uint32_t tl = tmem_base + (static_cast<uint32_t>(q4 * 32) << 16);
+    int q = 0;
+    uint32_t qphase = 0, j = 0;
     while (true) {
-      if (!consumer_all(warp_wait(qfull_bar(q), qphase, abort_p, a.status))) break;
+      if (!epi_all(warp_wait(qfull_bar(q), qphase, abort_p, a.status))) break;
       const UnitDesc ud = qdesc[q];
       __syncwarp();
       if (lane == 0) mbar_arrive(qempty_bar(q));
       if (++q == kDecQueue) { q = 0; qphase ^= 1u; }
-      if (ud.kind < 0) break;
-      bool ok = true;
-      // gate/up rows: warp w takes rows w, w + 8, ... of each stage
-      for (int st = 0; st < n13; ++st) {
-        if (!consumer_all(warp_wait(full_bar(stage), sphase, abort_p, a.status))) { ok = false; break; }
-        const uint8_t* tile = ring + stage * kDecStageBytes;
-        for (int rl = warp; rl < rs; rl += kDecWarps) {
-          const uint4* row = reinterpret_cast<const uint4*>(tile + rl * D * 2);
-          float wv[NV][8];
+      if (ud.kind < 0) break;  // the same descriptor in every warp
+      // D1 -> SwiGLU -> a^T (bf16, the B operand of the down MMAs)
+      if (!epi_all(warp_wait(gu_full, j & 1u, abort_p, a.status))) break;
+      tc_fence_after();
+      float z[kDecN];
+      tmem_ld16(tl, z);
+      tmem_ld_wait_regs16(z);
+      if (q4 >= 2) {
 #pragma unroll
-          for (int v = 0; v < NV; ++v) {
-            const uint4 x = row[v * 32 + lane];
-            wv[v][0] = bf_lo(x.x); wv[v][1] = bf_hi(x.x); wv[v][2] = bf_lo(x.y); wv[v][3] = bf_hi(x.y);
-            wv[v][4] = bf_lo(x.z); wv[v][5] = bf_hi(x.z); wv[v][6] = bf_lo(x.w); wv[v][7] = bf_hi(x.w);
-          }
-          for (int i = 0; i < ud.n_tok; ++i) {
-            const int t = ud.tok_off < 0 ? i : s_tok[ud.tok_off + i];
-            float acc = 0.0f;
+        for (int t = 0; t < kDecN; ++t) upx[r - 64][t] = z[t];
+      }
+      epi_sync();
+      if (q4 < 2) {
 #pragma unroll
-            for (int v = 0; v < NV; ++v) {
-              const float4* up = reinterpret_cast<const float4*>(uf + t * D + (v * 32 + lane) * 8);
-              const float4 p0 = up[0], p1 = up[1];
-              acc = fmaf(p0.x, wv[v][0], acc); acc = fmaf(p0.y, wv[v][1], acc);
-              acc = fmaf(p0.z, wv[v][2], acc); acc = fmaf(p0.w, wv[v][3], acc);
-              acc = fmaf(p1.x, wv[v][4], acc); acc = fmaf(p1.y, wv[v][5], acc);
-              acc = fmaf(p1.z, wv[v][6], acc); acc = fmaf(p1.w, wv[v][7], acc);
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) zbuf[st * rs + rl][i] = acc;
-          }
+        for (int t = 0; t < kDecN; ++t) {
+          const float av = t < T ? silu_mul(z[t], upx[r][t]) : 0.0f;
+          *reinterpret_cast<bf16*>(at + sw128_off(t, r)) = __float2bfloat16_rn(av);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty_bar(stage));
-        if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
       }
-      if (!ok) break;  // the same decision in every compute warp
-      consumer_sync();  // zbuf complete
-      // SwiGLU of the unit's 64 rows (packed block: gate rows 0-63, up 64-127)
-      for (int i = tid; i < kDecUC * ud.n_tok; i += kDecWarps * 32) {
-        const int j = i / ud.n_tok, tt = i - j * ud.n_tok;
-        abuf[j][tt] = silu_mul(zbuf[j][tt], zbuf[64 + j][tt]);
-      }
-      consumer_sync();
-      // partial down projection: thread r takes W2 row box*256 + r
-      for (int bx = 0; bx < n2; ++bx) {
-        if (!consumer_all(warp_wait(full_bar(stage), sphase, abort_p, a.status))) { ok = false; break; }
-        const uint8_t* tile = ring + stage * kDecStageBytes;
-        const int r = tid;  // 0 .. 255
-        const int jrow = bx * kDecW2Rows + r;
-        if (jrow < D) {
-          float wv[64];
+      fence_async_shared();  // a^T written by the generic proxy, read by the tensor cores
+      tc_fence_before();
+      epi_sync();
+      if (tid == 128) mbar_arrive(a_ready);
+      // D2 -> the unit's partial rows
+      if (!epi_all(warp_wait(dn_full, j & 1u, abort_p, a.status))) break;
+      tc_fence_after();
+      float* base = a.part + static_cast<int64_t>(ud.slot) * D + r;
+      for (int m = 0; m < MT2; ++m) {
+        float y[kDecN];
+        tmem_ld16(tl + kDecN + m * kDecN, y);
+        tmem_ld_wait_regs16(y);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            // 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r & 7)
-            const uint4 x = *reinterpret_cast<const uint4*>(tile + r * 128 + ((c ^ (r & 7)) << 4));
-            wv[c * 8 + 0] = bf_lo(x.x); wv[c * 8 + 1] = bf_hi(x.x);
-            wv[c * 8 + 2] = bf_lo(x.y); wv[c * 8 + 3] = bf_hi(x.y);
-            wv[c * 8 + 4] = bf_lo(x.z); wv[c * 8 + 5] = bf_hi(x.z);
-            wv[c * 8 + 6] = bf_lo(x.w); wv[c * 8 + 7] = bf_hi(x.w);
-          }
-          for (int i = 0; i < ud.n_tok; ++i) {
-            float acc = 0.0f;
-#pragma unroll
-            for (int k = 0; k < kDecUC; ++k) acc = fmaf(wv[k], abuf[k][i], acc);
-            a.part[static_cast<int64_t>(ud.slot + i) * D + jrow] = acc;
-          }
+        for (int t = 0; t < kDecN; ++t) {
+          const int row = ud.row_of[t];
+          if (row >= 0) base[static_cast<int64_t>(row) * D + m * 128] = y[t];
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty_bar(stage));
-        if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
       }
-      if (!ok) break;
-      __threadfence();  // this thread's partials, before the unit is counted
-      consumer_sync();
-      if (tid == 0) atomicAdd(&a.sync->units_done, 1);
+      __threadfence();  // the partials, before the unit is counted
+      tc_fence_before();
+      epi_sync();
+      if (tid == 128) atomicAdd(&a.sync->units_done, 1);
+      ++j;
     }
   }
 
   // ---- 3. combine ------------------------------------------------------------
+  tc_fence_before();
   __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kDecTmemCols);
+  }
   if (*abort_p) {
     record_status(a.status, MOE_ERR_DEVICE_CHECK);
     return;
@@ -506,54 +557,65 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW2, const __grid_const
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // one warp per (token, 4 columns): the lanes share the token's partial
+  // rows (shared units with gate 1, then each routed slot's chunks with its
+  // gate), each lane in a fixed order, then a fixed shuffle tree
   const int cols4 = D / 4;
-  for (int g = blockIdx.x * kDecThreads + tid; g < T * cols4; g += gridDim.x * kDecThreads) {
-    const int t = g / cols4;
-    const int col = (g - t * cols4) * 4;
-    const uint2 uv = *reinterpret_cast<const uint2*>(a.u + static_cast<int64_t>(t) * D + col);
-    float4 acc = make_float4(bf_lo(uv.x), bf_hi(uv.x), bf_lo(uv.y), bf_hi(uv.y));
-    float4 sh = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int su = 0; su < S; ++su) {
-      const float4 p = __ldcg(reinterpret_cast<const float4*>(
-          a.part + static_cast<int64_t>(su * T + t) * D + col));
-      sh.x += p.x; sh.y += p.y; sh.z += p.z; sh.w += p.w;
-    }
-    acc.x += sh.x; acc.y += sh.y; acc.z += sh.z; acc.w += sh.w;
-    for (int k = 0; k < K; ++k) {
-      const int e = s_idx[t * K + k];
-      const int cnt = s_cnt[e];
-      const int64_t base = static_cast<int64_t>(S) * T + static_cast<int64_t>(s_off[e]) * nc +
-                           s_rank[t * K + k];
-      float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int c = 0; c < nc; ++c) {
-        const float4 p = __ldcg(reinterpret_cast<const float4*>(
-            a.part + (base + static_cast<int64_t>(c) * cnt) * D + col));
-        y.x += p.x; y.y += p.y; y.z += p.z; y.w += p.w;
+  const int R = S + K * nc;
+  const int gwarps = static_cast<int>(gridDim.x) * (kDecThreads / 32);
+  for (int item = static_cast<int>(blockIdx.x) * (kDecThreads / 32) + warp; item < T * cols4;
+       item += gwarps) {
+    const int t = item / cols4;
+    const int col = (item - t * cols4) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int jr = lane; jr < R; jr += 32) {
+      int64_t row;
+      float g;
+      if (jr < S) {
+        row = static_cast<int64_t>(jr) * T + t;
+        g = 1.0f;
+      } else {
+        const int kk = (jr - S) / nc, c = (jr - S) - kk * nc;
+        const int e = s_idx[t * K + kk];
+        row = static_cast<int64_t>(S) * T + static_cast<int64_t>(s_off[e]) * nc +
+              static_cast<int64_t>(c) * s_cnt[e] + s_rank[t * K + kk];
+        g = __ldcg(a.w + t * K + kk);
       }
-      const float wk = __ldcg(a.w + t * K + k);
-      acc.x = fmaf(wk, y.x, acc.x); acc.y = fmaf(wk, y.y, acc.y);
-      acc.z = fmaf(wk, y.z, acc.z); acc.w = fmaf(wk, y.w, acc.w);
+      const float4 p = __ldcg(reinterpret_cast<const float4*>(a.part + row * D + col));
+      acc.x = fmaf(g, p.x, acc.x); acc.y = fmaf(g, p.y, acc.y);
+      acc.z = fmaf(g, p.z, acc.z); acc.w = fmaf(g, p.w, acc.w);
     }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 o;
-    o.x = *reinterpret_cast<uint32_t*>(&lo);
-    o.y = *reinterpret_cast<uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(a.h + static_cast<int64_t>(t) * D + col) = o;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+      acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+      acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+      acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+    }
+    if (lane == 0) {
+      const uint2 uv = *reinterpret_cast<const uint2*>(a.u + static_cast<int64_t>(t) * D + col);
+      __nv_bfloat162 lo = __floats2bfloat162_rn(bf_lo(uv.x) + acc.x, bf_hi(uv.x) + acc.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(bf_lo(uv.y) + acc.z, bf_hi(uv.y) + acc.w);
+      uint2 o;
+      o.x = *reinterpret_cast<uint32_t*>(&lo);
+      o.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(a.h + static_cast<int64_t>(t) * D + col) = o;
+    }
   }
 }
 
-
-constexpr int dec_smem_bytes(int D) { return 1024 + kDecStages * kDecStageBytes + kDecMaxT * D * 4; }
+constexpr int dec_smem_bytes(int D) {
+  return 1024 + kDecStages * kDecTileBytes + (D / 64) * kDecN * 128 + kDecN * 128;
+}
 
 template <int NV>
-int launch_decode_nv(const CUtensorMap& m2, const CUtensorMap& m2s, const DecArgs& a, int grid,
-                     cudaStream_t st) {
+int launch_decode_nv(const CUtensorMap& m13, const CUtensorMap& m13s, const CUtensorMap& m2,
+                     const CUtensorMap& m2s, const DecArgs& a, int grid, cudaStream_t st) {
   static std::atomic<uint64_t> optin{0};
   auto kern = decode_layer_kernel<NV>;
   const int smem = dec_smem_bytes(NV * 256);
   if (int rc = ensure_smem_optin(reinterpret_cast<const void*>(kern), smem, optin)) return rc;
-  return launch_k(kern, grid, kDecThreads, smem, st, 1, m2, m2s, a);
+  return launch_k(kern, grid, kDecThreads, smem, st, 1, m13, m13s, m2, m2s, a);
 }
 
 }  // namespace
@@ -577,15 +639,18 @@ int launch_decode_fused(const moe_shape_t& s, const void* u, const void* E, cons
                         void* h, int32_t* idx, float* w, float* logits, float* part, void* sync,
                         int32_t* status, int sms, cudaStream_t st) {
   const uint64_t d = static_cast<uint64_t>(s.d), I = static_cast<uint64_t>(s.inter);
-  CUtensorMap m2, m2s;
-  if (!make_map_2d(&m2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W2, I,
-                   static_cast<uint64_t>(s.n_routed) * d, I * 2, kDecUC, kDecW2Rows))
+  const uint64_t n = static_cast<uint64_t>(s.n_routed), ks = static_cast<uint64_t>(s.n_shared);
+  CUtensorMap m13, m13s, m2, m2s;
+  if (!make_map_2d(&m13, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W13, d, n * 2 * I, d * 2, 64, 128) ||
+      !make_map_2d(&m2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W2, I, n * d, I * 2, 64, 128))
     return MOE_ERR_CUDA;
-  if (s.n_shared > 0) {
-    if (!make_map_2d(&m2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W2_s, I,
-                     static_cast<uint64_t>(s.n_shared) * d, I * 2, kDecUC, kDecW2Rows))
+  if (ks > 0) {
+    if (!make_map_2d(&m13s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W13_s, d, ks * 2 * I, d * 2, 64,
+                     128) ||
+        !make_map_2d(&m2s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W2_s, I, ks * d, I * 2, 64, 128))
       return MOE_ERR_CUDA;
   } else {
+    m13s = m13;
     m2s = m2;
   }
   if (cudaMemsetAsync(sync, 0, sizeof(DecSync), st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -593,8 +658,6 @@ int launch_decode_fused(const moe_shape_t& s, const void* u, const void* E, cons
   a.u = static_cast<const bf16*>(u);
   a.E = static_cast<const bf16*>(E);
   a.bias = bias;
-  a.W13 = static_cast<const bf16*>(W13);
-  a.W13_s = static_cast<const bf16*>(W13_s);
   a.h = static_cast<bf16*>(h);
   a.idx = idx;
   a.w = w;
@@ -610,10 +673,10 @@ int launch_decode_fused(const moe_shape_t& s, const void* u, const void* E, cons
   a.K = s.top_k;
   a.flags = s.flags;
   switch (s.d) {
-    case 256: return launch_decode_nv<1>(m2, m2s, a, sms, st);
-    case 512: return launch_decode_nv<2>(m2, m2s, a, sms, st);
-    case 1024: return launch_decode_nv<4>(m2, m2s, a, sms, st);
-    case 2048: return launch_decode_nv<8>(m2, m2s, a, sms, st);
+    case 256: return launch_decode_nv<1>(m13, m13s, m2, m2s, a, sms, st);
+    case 512: return launch_decode_nv<2>(m13, m13s, m2, m2s, a, sms, st);
+    case 1024: return launch_decode_nv<4>(m13, m13s, m2, m2s, a, sms, st);
+    case 2048: return launch_decode_nv<8>(m13, m13s, m2, m2s, a, sms, st);
     default: return MOE_ERR_SHAPE;
   }
 }

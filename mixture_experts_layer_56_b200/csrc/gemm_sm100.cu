@@ -369,17 +369,19 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool make_map_bf16(CUtensorMap* map, int rank, const void* base, uint64_t inner, uint64_t rows,
                    uint64_t depth, uint64_t row_stride_bytes, uint64_t depth_stride_bytes,
-                   uint32_t box_rows) {
+                   uint32_t box_rows, uint32_t box_k) {
   auto fn = encode_fn();
   if (!fn || !base || inner == 0 || rows == 0 || depth == 0 || (rank != 2 && rank != 3))
     return false;
   if (rank == 2 && depth != 1) return false;
   cuuint64_t dims[3] = {inner, rows, depth};
   cuuint64_t strides[2] = {row_stride_bytes, depth_stride_bytes};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), box_rows, 1};
+  if (box_k != 64 && box_k != 32) return false;
+  cuuint32_t box[3] = {box_k, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult res = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims,
-                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    box_k == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return res == CUDA_SUCCESS;
 }

@@ -60,9 +60,11 @@ struct GemmMaps {
   CUtensorMap a_r, a_s, b_r, b_s;
 };
 
+// box_k: 64 (128-byte rows, 128-byte swizzle) or 32 (64-byte rows, 64-byte
+// swizzle).
 bool make_map_bf16(CUtensorMap* map, int rank, const void* base, uint64_t inner, uint64_t rows,
                    uint64_t depth, uint64_t row_stride_bytes, uint64_t depth_stride_bytes,
-                   uint32_t box_rows);
+                   uint32_t box_rows, uint32_t box_k = 64);
 
 // Rank-2 map with 128-byte swizzle: box {box_inner, box_rows}; the box's
 // inner extent must be 128 bytes.
@@ -74,8 +76,10 @@ int launch_grouped_gemm(int BN, int epi, const GemmMaps& maps, const GroupedGemm
 
 // The same GEMM on 2-CTA clusters with 256-row tiles (gemm_sm100_pair.cu).
 // B maps must have box rows BN / 2 (128 for BN = 512, the wide tiles of
-// 256 x 512 whose B rows come in two 128-row boxes per k-block).  `clusters`
-// CTA pairs are launched.
+// 256 x 512 whose B rows come in two 128-row boxes per k-block).  The wide
+// tiles step through K in blocks of kWideBK (maps with box_k = kWideBK; the
+// args' k-block counts in those units).  `clusters` CTA pairs are launched.
+constexpr int kWideBK = 32;
 int launch_grouped_gemm_pair(int BN, int epi, const GemmMaps& maps, const GroupedGemmArgs& args,
                              int clusters, cudaStream_t stream);
 

@@ -440,26 +440,39 @@ constexpr int kWideBN = 512;
 constexpr int kWideHalf = 256;
 constexpr int kWideEpiWarps = 8;
 
+// k-blocks of kWideBK = 32 (64-byte rows, 64-byte swizzle): 24 KB stages,
+// so that more of them, 7, are in flight at once.  One stage's MMAs take
+// 512 clocks of tensor work, and a TMA load takes about 3000 clocks to land
+// under full load (the pipe utilisation of 3-stage 48 KB and 5-stage 32 KB
+// rings both fit that), so about 7 stages keep the pipe fed.
+template <int BKW>
+constexpr int wide_stage_bytes() {
+  return HBM_ROWS * BKW * 2 + (kWideBN / 2) * BKW * 2;
+}
+template <int BKW>
 constexpr int wide_stages() {
-  return (216 * 1024 - kWideEpiWarps * kWarpStageBytes) /
-         (HBM_ROWS * PBK * 2 + (kWideBN / 2) * PBK * 2);
+  return (216 * 1024 - kWideEpiWarps * kWarpStageBytes) / wide_stage_bytes<BKW>();
 }
-
+template <int BKW>
 constexpr int wide_smem_bytes() {
-  return wide_stages() * (HBM_ROWS * PBK * 2 + (kWideBN / 2) * PBK * 2) +
-         kWideEpiWarps * kWarpStageBytes + 1024;
+  return wide_stages<BKW>() * wide_stage_bytes<BKW>() + kWideEpiWarps * kWarpStageBytes + 1024;
 }
 
-template <int EPI>
+template <int BKW>
+__device__ __forceinline__ uint64_t wide_desc(uint32_t saddr) {
+  return BKW == 64 ? desc_kmajor_sw128(saddr) : desc_kmajor_sw64(saddr);
+}
+
+template <int EPI, int BKW>
 __global__ void __launch_bounds__(kPairThreads, 1)
 grouped_gemm_pair_wide_kernel(const __grid_constant__ CUtensorMap tmA_r,
                               const __grid_constant__ CUtensorMap tmA_s,
                               const __grid_constant__ CUtensorMap tmB_r,
                               const __grid_constant__ CUtensorMap tmB_s,
                               const GroupedGemmArgs args) {
-  constexpr int STAGES = wide_stages();
-  constexpr uint32_t A_BYTES = HBM_ROWS * PBK * 2;
-  constexpr uint32_t BH_BYTES = 128 * PBK * 2;  // this CTA's rows of one 256-column slice
+  constexpr int STAGES = wide_stages<BKW>();
+  constexpr uint32_t A_BYTES = HBM_ROWS * BKW * 2;
+  constexpr uint32_t BH_BYTES = 128 * BKW * 2;  // this CTA's rows of one 256-column slice
   constexpr uint32_t STAGE_BYTES = A_BYTES + 2 * BH_BYTES;
   constexpr uint32_t TMEM_COLS = 512;
   constexpr uint32_t IDESC = idesc_bf16_f32(PBM, kWideHalf);
@@ -588,10 +601,10 @@ grouped_gemm_pair_wide_kernel(const __grid_constant__ CUtensorMap tmA_r,
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_p, args.status)) { ok = false; break; }
           const uint32_t sa = smem_base + stage * STAGE_BYTES;
           const uint32_t fb = leader ? full_bar(stage) : map_to_cta(full_bar(stage), 0);
-          const int kx = (kb % args.kb_per_expert) * PBK;
+          const int kx = (kb % args.kb_per_expert) * BKW;
           const int kz = zbase + kb / args.kb_per_expert;
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-          tma_load_2d_pair(sa, ma, fb, kb * PBK, row);
+          tma_load_2d_pair(sa, ma, fb, kb * BKW, row);
           tma_load_3d_pair(sa + A_BYTES, mb, fb, kx, nrow, kz);
           tma_load_3d_pair(sa + A_BYTES + BH_BYTES, mb, fb, kx, nrow + kWideHalf, kz);
           issued |= 1u << stage;
@@ -636,9 +649,9 @@ grouped_gemm_pair_wide_kernel(const __grid_constant__ CUtensorMap tmA_r,
             }
             const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(h * kWideHalf);
 #pragma unroll
-            for (int k = 0; k < PBK / 16; ++k) {
-              mma_bf16_pair(d_tmem, desc_kmajor_sw128(sa + k * 32),
-                            desc_kmajor_sw128(sb + h * BH_BYTES + k * 32), IDESC,
+            for (int k = 0; k < BKW / 16; ++k) {
+              mma_bf16_pair(d_tmem, wide_desc<BKW>(sa + k * 32),
+                            wide_desc<BKW>(sb + h * BH_BYTES + k * 32), IDESC,
                             (kb > 0 || k > 0) ? 1u : 0u);
             }
             if (kb == nkb - 1) mma_commit_pair(tfull_bar(h), kBoth);
@@ -773,11 +786,11 @@ template <int EPI>
 int launch_wide_impl(const GemmMaps& m, const GroupedGemmArgs& args, int clusters,
                      cudaStream_t stream) {
   static std::atomic<uint64_t> optin{0};
-  auto kern = grouped_gemm_pair_wide_kernel<EPI>;
-  if (int rc = ensure_smem_optin(reinterpret_cast<const void*>(kern), wide_smem_bytes(), optin))
-    return rc;
-  return launch_k(kern, dim3(2 * clusters), kPairThreads, wide_smem_bytes(), stream, 2, m.a_r,
-                  m.a_s, m.b_r, m.b_s, args);
+  auto kern = grouped_gemm_pair_wide_kernel<EPI, kWideBK>;
+  constexpr int smem = wide_smem_bytes<kWideBK>();
+  if (int rc = ensure_smem_optin(reinterpret_cast<const void*>(kern), smem, optin)) return rc;
+  return launch_k(kern, dim3(2 * clusters), kPairThreads, smem, stream, 2, m.a_r, m.a_s, m.b_r,
+                  m.b_s, args);
 }
 
 template <int BN, int EPI>

@@ -201,13 +201,17 @@ __global__ void __launch_bounds__(kSgThreads)
 dispatch_scatter_gather_kernel(const int32_t* __restrict__ idx, int64_t T, int K, int n,
                                const int32_t* __restrict__ chunk_base, int32_t* __restrict__ perm,
                                int32_t* __restrict__ inv, const TE* __restrict__ u, int d,
-                               TE* __restrict__ xperm) {
+                               TE* __restrict__ xperm, int parts) {
+  // `parts` blocks share a chunk: each ranks the chunk's tokens (cheap), the
+  // first of them writes perm / inv, and each copies every parts-th row
   __shared__ int wc[kDispWarps][256];
   __shared__ int spos[kDispatchChunk][KMAX];
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kDispatchChunk;
+  const int chunk = static_cast<int>(blockIdx.x) / parts;
+  const int part = static_cast<int>(blockIdx.x) - chunk * parts;
+  const int64_t t0 = static_cast<int64_t>(chunk) * kDispatchChunk;
   const bool ranker = warp < kDispWarps;  // warp-uniform
   const int64_t t = t0 + threadIdx.x;
   int ek[KMAX];
@@ -226,7 +230,7 @@ dispatch_scatter_gather_kernel(const int32_t* __restrict__ idx, int64_t T, int K
   }
   __syncthreads();
   for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    int run = chunk_base[static_cast<int64_t>(blockIdx.x) * n + e];
+    int run = chunk_base[static_cast<int64_t>(chunk) * n + e];
     for (int w = 0; w < kDispWarps; ++w) {
       const int c = wc[w][e];
       wc[w][e] = run;
@@ -250,21 +254,24 @@ dispatch_scatter_gather_kernel(const int32_t* __restrict__ idx, int64_t T, int K
           for (int k = 0; k < KMAX; ++k)
             if (ek[k] == e) kk = k;
           const int64_t slot = t * K + kk;
-          perm[pos] = static_cast<int32_t>(slot);
-          inv[slot] = pos;
+          if (part == 0) {
+            perm[pos] = static_cast<int32_t>(slot);
+            inv[slot] = pos;
+          }
           spos[threadIdx.x][kk] = pos;
         }
       }
     }
   }
   __syncthreads();
-  // copy: warp w takes the chunk's tokens w, w + 16, ...
+  // copy: warp w of part p takes the chunk's tokens p * 16 + w, + 16 * parts, ...
   constexpr int V = Vec16<TE>::N;
   constexpr int U = kSgCopyUnroll;
+  constexpr int W = kSgThreads / 32;
   const int nv = d / V;
   const int64_t rem = T - t0;
   const int nt = rem < kDispatchChunk ? static_cast<int>(rem) : kDispatchChunk;
-  for (int tl = warp; tl < nt; tl += kSgThreads / 32) {
+  for (int tl = part * W + warp; tl < nt; tl += W * parts) {
     const uint4* src = reinterpret_cast<const uint4*>(u + (t0 + tl) * static_cast<int64_t>(d));
     for (int c0 = lane; c0 < nv; c0 += 32 * U) {
       uint4 v[U];
@@ -699,13 +706,17 @@ int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_
                         nch, n, chunk_base, counts, offsets))
     return r2;
   if (dg && dg->xperm) {
-    // scatter and gather in one launch
+    // scatter and gather in one launch; enough blocks share each chunk's
+    // copies that the grid covers every SM about twice
     const int bf = dg->dtype == MOE_DTYPE_BF16;
+    const int64_t want = (2 * 148 + nch - 1) / nch;
+    const int parts = static_cast<int>(want < 1 ? 1 : (want > 8 ? 8 : want));
+    const dim3 sg_grid(static_cast<unsigned>(nch * parts));
     rc = MOE_ERR_SHAPE;
 #define MOE_SG_LAUNCH(W, KM, TE)                                                             \
-  launch_k(dispatch_scatter_gather_kernel<W, KM, TE>, grid, kSgThreads, 0, st, 1, idx, T, K, n, \
-           static_cast<const int32_t*>(chunk_base), perm, inv, static_cast<const TE*>(dg->u),   \
-           dg->d, static_cast<TE*>(dg->xperm))
+  launch_k(dispatch_scatter_gather_kernel<W, KM, TE>, sg_grid, kSgThreads, 0, st, 1, idx, T, K, \
+           n, static_cast<const int32_t*>(chunk_base), perm, inv, static_cast<const TE*>(dg->u), \
+           dg->d, static_cast<TE*>(dg->xperm), parts)
 #define MOE_SG_CASE(W)                                                                       \
   case W:                                                                                    \
     rc = bf ? (K <= 8 ? MOE_SG_LAUNCH(W, 8, bf16)                                            \

@@ -39,6 +39,9 @@ from mixture_experts_layer_56_b200.layer import MoELayer, to_device, to_numpy
 from oracle import moe_oracle as O
 
 TIE_GAP = 1e-5
+PATH_NAMES = {L.MOE_PATH_STAGES: "stages (bit-equal to the stage-wise calls)",
+              L.MOE_PATH_DECODE_LAYER: "decode layer kernel",
+              L.MOE_PATH_SMALL_BATCH: "small-batch front kernel + grouped GEMMs + combine"}
 NAMES = ("u", "E", "bias", "W1", "W3", "W2", "W1_s", "W3_s", "W2_s")
 
 
@@ -98,7 +101,7 @@ def check_forward(gpu: dict, ref_h: np.ndarray, near: np.ndarray, bf16: bool, to
         return None
     keep = ~near if tokens is None else ~near[tokens]
     assert keep.any(), "every token is a near tie: the case checks nothing"
-    assert_close(h_fwd[keep], ref_h[keep], "h (decode layer kernel)", bf16)
+    assert_close(h_fwd[keep], ref_h[keep], f"h (forward path {gpu['path']})", bf16)
     return error_stats(h_fwd[keep], ref_h[keep], bf16)
 
 
@@ -257,8 +260,7 @@ def full_parity(x: S.LayerInputs, flags: int = 0, device="cuda:0"):
     eh = assert_close(gpu["h"], ref_h, "h", bf16)
     fwd = check_forward(gpu, ref_h, O.topk_gap(key, wl.top_k) < TIE_GAP, bf16)
     rep = dict(workload=wl.name, tokens=int(wl.T), tokens_checked=int(wl.T), flags=int(flags),
-               forward_path=("decode layer kernel" if gpu["path"] == L.MOE_PATH_DECODE_LAYER
-                             else "stages (bit-equal to the stage-wise calls)"),
+               forward_path=PATH_NAMES[gpu["path"]],
                h_forward=fwd,
                near_ties=near, mismatches=mism, err_y=ey, err_ysh=esh, err_h=eh,
                h=error_stats(gpu["h"], ref_h, bf16), y=error_stats(gpu["y"], ref["y"], bf16),
@@ -311,8 +313,7 @@ def sampled_parity(x: S.LayerInputs, device="cuda:0", n_random: int = 512):
     esh = assert_close(gpu["ysh"][toks], ref_sh, "ysh (sampled)")
     fwd = check_forward(gpu, ref_h, O.topk_gap(s, wl.top_k) < TIE_GAP, True, tokens=toks)
     rep = dict(workload=wl.name, tokens=int(wl.T), tokens_checked=int(toks.size), flags=0,
-               forward_path=("decode layer kernel" if gpu["path"] == L.MOE_PATH_DECODE_LAYER
-                             else "stages (bit-equal to the stage-wise calls)"),
+               forward_path=PATH_NAMES[gpu["path"]],
                h_forward=fwd,
                near_ties=near, mismatches=mism, err_h=eh, err_ysh=esh, sampled=int(toks.size),
                h=error_stats(gpu["h"][toks], ref_h), ysh=error_stats(gpu["ysh"][toks], ref_sh),

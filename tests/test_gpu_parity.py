@@ -312,6 +312,8 @@ DECODE_CASES = [
     W("dec_d1024_noshared", T=5, d=1024, n_routed=32, n_shared=0, inter=256, top_k=3),
     W("dec_d2048_k16", T=3, d=2048, n_routed=256, n_shared=1, inter=64, top_k=16, bias_var=4.0),
     W("dec_d256_t7", T=7, d=256, n_routed=8, n_shared=4, inter=320, top_k=8),
+    W("dec_d1024_t16", T=16, d=1024, n_routed=40, n_shared=2, inter=128, top_k=6),
+    W("dec_d2048_t13", T=13, d=2048, n_routed=64, n_shared=2, inter=192, top_k=6, bias_var=0.5),
 ]
 
 
@@ -339,3 +341,52 @@ def test_decode_layer_kernel_select_only_bias_and_repeat():
     assert layer.status() == 0
     assert np.array_equal(h1, h2)
     assert np.array_equal(h1, rep["gpu"]["h_fwd_raw"])
+
+
+# Batches of 17 to 128 tokens route, dispatch and gather in one kernel before
+# the grouped GEMMs (moe_forward_path MOE_PATH_SMALL_BATCH).
+SMALL_BATCH_CASES = [
+    W("sb_t17", T=17, d=512, n_routed=64, n_shared=2, inter=128, top_k=6, bias_var=0.5),
+    W("sb_t100_n256", T=100, d=1024, n_routed=256, n_shared=1, inter=64, top_k=8),
+    W("sb_t128_noshared", T=128, d=256, n_routed=20, n_shared=0, inter=192, top_k=3),
+]
+
+
+@pytest.mark.parametrize("wl", SMALL_BATCH_CASES, ids=[c.name for c in SMALL_BATCH_CASES])
+def test_small_batch_front_kernel(wl):
+    x = S.make_inputs(wl)
+    rep = P.full_parity(x)
+    assert rep["gpu"]["path"] == L.MOE_PATH_SMALL_BATCH
+    assert rep["h_forward"] is not None
+
+
+@pytest.mark.parametrize("T", [4, 64])
+def test_small_paths_replay_from_a_cuda_graph_bitwise(T):
+    """The one-kernel decode layer (T = 4) and the small-batch front kernel
+    (T = 64) zero their sync words with a memset node before the kernel:
+    captured into a CUDA graph, every replay gives the eager result."""
+    wl = W(f"graph{T}", T=T, d=512, n_routed=32, n_shared=1, inter=128, top_k=4)
+    x = S.make_inputs(wl)
+    layer = MoELayer(x)
+    assert L.moe_forward_path(layer.shape) == (L.MOE_PATH_DECODE_LAYER if T <= 16
+                                               else L.MOE_PATH_SMALL_BATCH)
+    u = to_device(x.u, "cuda:0")
+    h = torch.empty_like(u)
+
+    def fwd():
+        L.moe_layer_forward(layer.shape, u, layer.E, layer.bias, layer.W13, layer.W2,
+                            layer.W13_s, layer.W2_s, h, layer.ws,
+                            stream=torch.cuda.current_stream())
+
+    fwd()
+    torch.cuda.synchronize()
+    ref = to_numpy(h).copy()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd()
+    for _ in range(3):
+        h.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(to_numpy(h), ref)
+    assert layer.status() == 0
