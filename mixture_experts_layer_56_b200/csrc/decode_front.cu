@@ -4,22 +4,20 @@
 //
 // At a hundred tokens the three stages are latency chains, not bandwidth:
 // the logits are 2 T d N_r FLOPs, the dispatch a few hundred slots.  Here
-// they run on many SMs at once with two grid-wide steps in between:
-//  A. logits: each CTA takes (8 experts) x (8 tokens) items; warp w holds
-//     expert row e in registers, each lane 8 columns per 256, and forms
-//     u_t . e_i as one fp32 FMA chain per lane plus a fixed shuffle tree;
-//  B. after every item is written: softmax and top-K, one warp per token
-//     (lower expert index first on ties, gates not renormalised), written to
-//     idx / w;
-//  C. after every token is selected: each CTA builds the stable counting
-//     sort of the T*K slots (warp ballots per 32 tokens, as the one-block
+// they run on one CTA per token with a single grid-wide step:
+//  A/B. CTA c routes token c (and c + G, ...): the token's row in registers,
+//     warp w forms u_t . e_i for experts w, w + 8, ... as one fp32 FMA chain
+//     per lane plus a fixed shuffle tree, into shared memory; warp 0 then
+//     runs softmax and top-K (lower expert index first on ties, gates not
+//     renormalised) and writes idx / w;
+//  C. after every token is routed: each CTA builds the stable counting sort
+//     of the T*K slots (warp ballots per 32 tokens, as the one-block
 //     dispatch does), CTA 0 writes counts / offsets / perm / inv, and CTA c
-//     copies the rows of tokens c, c + G, ... of u to their K positions of
-//     X_perm.
-// The grid is at most one CTA per SM, so all of it is resident; the two
-// grid-wide steps are counters in the workspace (zeroed before the launch)
-// with bounded waits.  Results equal moe_route + moe_dispatch + the gather
-// up to the fp32 summation order of the logits.
+//     copies its tokens' rows of u to their K positions of X_perm.
+// The grid is at most one CTA per SM, so all of it is resident; the grid-wide
+// step is a counter in the workspace (zeroed before the launch) with a
+// bounded wait.  Results equal moe_route + moe_dispatch + the gather up to
+// the fp32 summation order of the logits.
 #include <cuda.h>
 #include <math_constants.h>
 
@@ -36,13 +34,10 @@ using namespace sm100;
 
 constexpr int kFrWarps = 8;
 constexpr int kFrThreads = kFrWarps * 32;
-constexpr int kFrTokens = 8;    // tokens per logits item
-constexpr int kFrExperts = 8;   // experts per logits item (one per warp)
 constexpr unsigned kFull = 0xffffffffu;
 
 struct FrontSync {
-  int logits_done;  // CTAs done with their logits items
-  int select_done;  // CTAs done with their tokens' selection
+  int select_done;  // CTAs done with their tokens' routing
 };
 
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
@@ -91,45 +86,40 @@ decode_front_kernel(const bf16* __restrict__ u, const bf16* __restrict__ E,
   pdl_wait();
   pdl_trigger();
 
-  // ---- A. logits -----------------------------------------------------------
-  const int n_eg = (n + kFrExperts - 1) / kFrExperts;
-  const int n_tb = (T + kFrTokens - 1) / kFrTokens;
-  for (int item = blockIdx.x; item < n_eg * n_tb; item += G) {
-    const int eg = item % n_eg, tb = item / n_eg;
-    const int e = eg * kFrExperts + warp;
-    if (e >= n) continue;  // warp-uniform
-    const uint4* er = reinterpret_cast<const uint4*>(E + static_cast<int64_t>(e) * D);
-    float ev[NV][8];
+  // ---- A. logits and B. softmax / top-K, one CTA per token ------------------
+  __shared__ float s_logit[256];
+  const bool select_only = (flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
+  for (int t = blockIdx.x; t < T; t += G) {
+    // the token's row stays in registers; warp w takes experts w, w + 8, ...,
+    // two expert rows in flight at a time
+    const uint4* ur = reinterpret_cast<const uint4*>(u + static_cast<int64_t>(t) * D);
+    uint4 uv[NV];
 #pragma unroll
-    for (int v = 0; v < NV; ++v) {
-      const uint4 x = er[v * 32 + lane];
-      ev[v][0] = bf_lo(x.x); ev[v][1] = bf_hi(x.x); ev[v][2] = bf_lo(x.y); ev[v][3] = bf_hi(x.y);
-      ev[v][4] = bf_lo(x.z); ev[v][5] = bf_hi(x.z); ev[v][6] = bf_lo(x.w); ev[v][7] = bf_hi(x.w);
-    }
-    const int t_beg = tb * kFrTokens;
-    const int t_end = min(T, t_beg + kFrTokens);
-    for (int t = t_beg; t < t_end; t += 2) {
-      // two tokens per pass: their row loads are in flight together
-      const bool two = t + 1 < t_end;
-      const uint4* ur0 = reinterpret_cast<const uint4*>(u + static_cast<int64_t>(t) * D);
-      const uint4* ur1 = reinterpret_cast<const uint4*>(u + static_cast<int64_t>(two ? t + 1 : t) * D);
-      uint4 u0[NV], u1[NV];
+    for (int v = 0; v < NV; ++v) uv[v] = ur[v * 32 + lane];
+    for (int e0 = warp; e0 < n; e0 += 2 * kFrWarps) {
+      const int e1 = e0 + kFrWarps;
+      const uint4* er0 = reinterpret_cast<const uint4*>(E + static_cast<int64_t>(e0) * D);
+      const uint4* er1 = reinterpret_cast<const uint4*>(E + static_cast<int64_t>(e1 < n ? e1 : e0) * D);
+      uint4 x0[NV], x1[NV];
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        u0[v] = ur0[v * 32 + lane];
-        u1[v] = ur1[v * 32 + lane];
+        x0[v] = er0[v * 32 + lane];
+        x1[v] = er1[v * 32 + lane];
       }
       float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        a0 = fmaf(bf_lo(u0[v].x), ev[v][0], a0); a0 = fmaf(bf_hi(u0[v].x), ev[v][1], a0);
-        a0 = fmaf(bf_lo(u0[v].y), ev[v][2], a0); a0 = fmaf(bf_hi(u0[v].y), ev[v][3], a0);
-        a0 = fmaf(bf_lo(u0[v].z), ev[v][4], a0); a0 = fmaf(bf_hi(u0[v].z), ev[v][5], a0);
-        a0 = fmaf(bf_lo(u0[v].w), ev[v][6], a0); a0 = fmaf(bf_hi(u0[v].w), ev[v][7], a0);
-        a1 = fmaf(bf_lo(u1[v].x), ev[v][0], a1); a1 = fmaf(bf_hi(u1[v].x), ev[v][1], a1);
-        a1 = fmaf(bf_lo(u1[v].y), ev[v][2], a1); a1 = fmaf(bf_hi(u1[v].y), ev[v][3], a1);
-        a1 = fmaf(bf_lo(u1[v].z), ev[v][4], a1); a1 = fmaf(bf_hi(u1[v].z), ev[v][5], a1);
-        a1 = fmaf(bf_lo(u1[v].w), ev[v][6], a1); a1 = fmaf(bf_hi(u1[v].w), ev[v][7], a1);
+        const float u0 = bf_lo(uv[v].x), u1 = bf_hi(uv[v].x), u2 = bf_lo(uv[v].y),
+                    u3 = bf_hi(uv[v].y), u4 = bf_lo(uv[v].z), u5 = bf_hi(uv[v].z),
+                    u6 = bf_lo(uv[v].w), u7 = bf_hi(uv[v].w);
+        a0 = fmaf(u0, bf_lo(x0[v].x), a0); a0 = fmaf(u1, bf_hi(x0[v].x), a0);
+        a0 = fmaf(u2, bf_lo(x0[v].y), a0); a0 = fmaf(u3, bf_hi(x0[v].y), a0);
+        a0 = fmaf(u4, bf_lo(x0[v].z), a0); a0 = fmaf(u5, bf_hi(x0[v].z), a0);
+        a0 = fmaf(u6, bf_lo(x0[v].w), a0); a0 = fmaf(u7, bf_hi(x0[v].w), a0);
+        a1 = fmaf(u0, bf_lo(x1[v].x), a1); a1 = fmaf(u1, bf_hi(x1[v].x), a1);
+        a1 = fmaf(u2, bf_lo(x1[v].y), a1); a1 = fmaf(u3, bf_hi(x1[v].y), a1);
+        a1 = fmaf(u4, bf_lo(x1[v].z), a1); a1 = fmaf(u5, bf_hi(x1[v].z), a1);
+        a1 = fmaf(u6, bf_lo(x1[v].w), a1); a1 = fmaf(u7, bf_hi(x1[v].w), a1);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
@@ -137,73 +127,71 @@ decode_front_kernel(const bf16* __restrict__ u, const bf16* __restrict__ E,
         a1 += __shfl_xor_sync(kFull, a1, o);
       }
       if (lane == 0) {
-        logits[t * n + e] = a0;
-        if (two) logits[(t + 1) * n + e] = a1;
+        s_logit[e0] = a0;
+        if (e1 < n) s_logit[e1] = a1;
       }
     }
-  }
-  if (!grid_step(&sync->logits_done, G, status)) return;
-
-  // ---- B. softmax and top-K, one warp per token ------------------------------
-  const bool select_only = (flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
-  for (int t = blockIdx.x * kFrWarps + warp; t < T; t += G * kFrWarps) {
-    float lg[8], key[8], ex[8];
-    float m = -CUDART_INF_F;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int e = lane + 32 * q;
-      float l = -CUDART_INF_F, kv = -CUDART_INF_F;
-      if (e < n) {
-        const float raw = __ldcg(logits + t * n + e);
-        kv = raw + (bias ? bias[e] : 0.0f);
-        l = select_only ? raw : kv;
-      }
-      lg[q] = l;
-      key[q] = kv;
-      m = fmaxf(m, l);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-    float z = 0.0f;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      ex[q] = (lane + 32 * q < n) ? expf(lg[q] - m) : 0.0f;
-      z += ex[q];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
-    const float inv_z = 1.0f / z;
-    unsigned taken = 0;
-    for (int k = 0; k < K; ++k) {
-      float bv = -CUDART_INF_F;
-      int bi = 0x7fffffff;
+    __syncthreads();
+    if (warp == 0) {
+      float lg[8], key[8], ex[8];
+      float m = -CUDART_INF_F;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int e = lane + 32 * q;
-        if (!((taken >> q) & 1u) && e < n && (key[q] > bv || bi == 0x7fffffff)) {
-          bv = key[q];
-          bi = e;
+        float l = -CUDART_INF_F, kv = -CUDART_INF_F;
+        if (e < n) {
+          const float raw = s_logit[e];
+          kv = raw + (bias ? bias[e] : 0.0f);
+          l = select_only ? raw : kv;
         }
+        lg[q] = l;
+        key[q] = kv;
+        m = fmaxf(m, l);
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(kFull, bv, o);
-        const int oi = __shfl_xor_sync(kFull, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if ((bi & 31) == lane) {
-        taken |= 1u << (bi >> 5);
-        float g = 0.0f;
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+      float z = 0.0f;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q == (bi >> 5)) g = ex[q];
-        idx[t * K + k] = bi;
-        w[t * K + k] = g * inv_z;
+      for (int q = 0; q < 8; ++q) {
+        ex[q] = (lane + 32 * q < n) ? expf(lg[q] - m) : 0.0f;
+        z += ex[q];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
+      const float inv_z = 1.0f / z;
+      unsigned taken = 0;
+      for (int k = 0; k < K; ++k) {
+        float bv = -CUDART_INF_F;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int e = lane + 32 * q;
+          if (!((taken >> q) & 1u) && e < n && (key[q] > bv || bi == 0x7fffffff)) {
+            bv = key[q];
+            bi = e;
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(kFull, bv, o);
+          const int oi = __shfl_xor_sync(kFull, bi, o);
+          if (ov > bv || (ov == bv && oi < bi)) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        if ((bi & 31) == lane) {
+          taken |= 1u << (bi >> 5);
+          float g = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (q == (bi >> 5)) g = ex[q];
+          idx[t * K + k] = bi;
+          w[t * K + k] = g * inv_z;
+        }
       }
     }
+    __syncthreads();  // s_logit is free for the next token
   }
   if (!grid_step(&sync->select_done, G, status)) return;
 
@@ -306,13 +294,14 @@ decode_front_kernel(const bf16* __restrict__ u, const bf16* __restrict__ E,
     }
   }
   __syncthreads();
-  // gather: warp w of CTA c copies tokens c * 8 + w, + 8 G, ...
-  for (int tt = blockIdx.x * kFrWarps + warp; tt < T; tt += G * kFrWarps) {
+  // gather: CTA c copies the rows of its tokens c, c + G, ...; warp w writes
+  // the copies k = w, w + 8, ...
+  for (int tt = blockIdx.x; tt < T; tt += G) {
     const uint4* src = reinterpret_cast<const uint4*>(u + static_cast<int64_t>(tt) * D);
     uint4 v[NV];
 #pragma unroll
     for (int j = 0; j < NV; ++j) v[j] = src[j * 32 + lane];
-    for (int kk = 0; kk < K; ++kk) {
+    for (int kk = warp; kk < K; kk += kFrWarps) {
       uint4* dst = reinterpret_cast<uint4*>(xperm + static_cast<int64_t>(spos[tt][kk]) * D);
 #pragma unroll
       for (int j = 0; j < NV; ++j) dst[j * 32 + lane] = v[j];
@@ -354,9 +343,7 @@ int launch_decode_front(const moe_shape_t& s, const void* u, const void* E, cons
                         int32_t* idx, float* w, float* logits, int32_t* counts, int32_t* offsets,
                         int32_t* perm, int32_t* inv, void* xperm, void* sync, int32_t* status,
                         int sms, cudaStream_t st) {
-  const int items = ((s.n_routed + kFrExperts - 1) / kFrExperts) *
-                    static_cast<int>((s.T + kFrTokens - 1) / kFrTokens);
-  const int grid = items < sms ? items : sms;
+  const int grid = s.T < sms ? static_cast<int>(s.T) : sms;
   if (cudaMemsetAsync(sync, 0, sizeof(FrontSync), st) != cudaSuccess) return MOE_ERR_CUDA;
   FrontSync* fs = static_cast<FrontSync*>(sync);
   switch (s.d) {

@@ -21,8 +21,11 @@
 //   store    the columns of the unit's own tokens (its expert's tokens, or all
 //            of them for a shared expert) as partial rows.
 // Roles (8 warps): warp 0 the TMA producer (unit counter, W13 and W2 tiles into
-// an 8-stage ring, running ahead into the next unit), warp 1 the MMA issuer,
-// warp 2 the TMEM owner, warps 4-7 the epilogue (TMEM lane quarters).
+// a 9-stage ring, running ahead into the next unit), warp 1 the MMA issuer,
+// warp 2 the TMEM owner, warps 4-7 the epilogue (TMEM lane quarters).  The
+// ring carries unit i's W13 tiles before unit i-1's W2 tiles, and D1 is
+// double-buffered, so unit i's gate/up MMAs run while the epilogue turns
+// unit i-1's D1 into a^T.
 //
 // Phases, all in this one launch (one CTA per SM):
 //  1. Router (CTAs 0 .. ceil(n/8)-1): logits u_t . e_i for 8 experts each,
@@ -57,11 +60,11 @@ constexpr int kDecThreads = 256;                     // 8 warps
 constexpr int kDecUC = 64;                           // intermediate rows per unit
 constexpr int kDecN = 16;                            // token columns of an MMA
 constexpr int kDecTileBytes = 128 * 64 * 2;          // one 128 x 64 bf16 TMA tile
-constexpr int kDecStages = 8;
+constexpr int kDecStages = 9;
 constexpr int kDecQueue = 4;                         // unit descriptors in flight
 constexpr int kDecRouterExperts = 8;                 // experts per router CTA
 constexpr int kDecMaxSlots = kDecMaxT * 32;          // routed (token, k) slots
-constexpr uint32_t kDecTmemCols = 512;               // D1 (16) + D2 (16 per 128 rows of d)
+constexpr uint32_t kDecTmemCols = 512;               // D1 (2 x 16) + D2 (16 per 128 rows of d)
 static_assert(kDecMaxT <= kDecN, "the batch fits one MMA's columns");
 
 // sync words of the decode scratch (zeroed before each launch)
@@ -241,10 +244,15 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
         ev[v][4] = bf_lo(x.z); ev[v][5] = bf_hi(x.z); ev[v][6] = bf_lo(x.w); ev[v][7] = bf_hi(x.w);
       }
       for (int t = 0; t < T; ++t) {
-        const uint4* ur = reinterpret_cast<const uint4*>(a.u + static_cast<int64_t>(t) * D);
+        // the token's row from the U tiles (16-byte chunk c of row t sits in
+        // tile c / 8 at chunk (c % 8) ^ (t % 8))
         uint4 uv[NV];
 #pragma unroll
-        for (int v = 0; v < NV; ++v) uv[v] = ur[v * 32 + lane];
+        for (int v = 0; v < NV; ++v) {
+          const int c = v * 32 + lane;
+          uv[v] = *reinterpret_cast<const uint4*>(ut + (c >> 3) * (kDecN * 128) +
+                                                  sw128_off(t, (c & 7) * 8));
+        }
         float acc = 0.0f;
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
@@ -348,15 +356,24 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
       uint32_t qphase = 0, sphase = 0;
       bool have_tables = false, ok = true;
       uint32_t issued = 0, issued_parity = 0;
+      int prev_kind = -1, prev_expert = 0, prev_chunk = 0;  // the unit whose W2 is due
       while (ok) {
         const int u = atomicAdd(&a.sync->unit_next, 1);
         if (u >= S && !have_tables) {
           // the routed units need the routing: build the expert tables
           if (!spin_until(&a.sync->route_done, 1, a.status)) { ok = false; break; }
           for (int e = 0; e < n; ++e) s_cnt[e] = 0;
+          // idx in batches of 16 independent loads, then the counting sort
+          for (int i0 = 0; i0 < T * K; i0 += 16) {
+            int v[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) v[jj] = i0 + jj < T * K ? __ldcg(a.idx + i0 + jj) : 0;
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+              if (i0 + jj < T * K) s_idx[i0 + jj] = v[jj];
+          }
           for (int i = 0; i < T * K; ++i) {
-            const int e = __ldcg(a.idx + i);
-            s_idx[i] = e;
+            const int e = s_idx[i];
             s_rank[i] = s_cnt[e]++;  // i runs in increasing t: ranks follow t
           }
           int run = 0, na = 0;
@@ -395,25 +412,34 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
         qdesc[q] = ud;
         mbar_arrive(qfull_bar(q));  // release: the descriptor and the tables
         if (++q == kDecQueue) { q = 0; qphase ^= 1u; }
-        if (ud.kind < 0) break;
-        // the unit's weights: its W13 block in KB13 tiles of 64 columns of d,
-        // then W2's rows in MT2 tiles of 128, columns chunk*64 .. +63
-        const CUtensorMap* m13 = ud.kind == 0 ? &tmW13s : &tmW13;
-        const CUtensorMap* m2 = ud.kind == 0 ? &tmW2s : &tmW2;
-        const int row13 = ud.expert * 2 * I + ud.chunk * 128;
-        for (int st = 0; st < KB13 + MT2 && ok; ++st) {
-          if (!wait_bounded(empty_bar(stage), sphase ^ 1u, abort_p, a.status)) { ok = false; break; }
+        // the ring order is W13(unit i), then W2(unit i-1): the MMAs of unit
+        // i's gate/up run while the epilogue turns unit i-1's into a^T
+        auto load = [&](const CUtensorMap* map, int x, int y) {
+          if (!wait_bounded(empty_bar(stage), sphase ^ 1u, abort_p, a.status)) return false;
           const uint32_t dst = ring_base + stage * kDecTileBytes;
           mbar_arrive_expect_tx(full_bar(stage), kDecTileBytes);
-          if (st < KB13)
-            tma_load_2d(dst, m13, full_bar(stage), st * 64, row13);
-          else
-            tma_load_2d(dst, m2, full_bar(stage), ud.chunk * kDecUC,
-                        ud.expert * D + (st - KB13) * 128);
+          tma_load_2d(dst, map, full_bar(stage), x, y);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (sphase << stage);
           if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
+          return true;
+        };
+        if (ud.kind >= 0) {
+          // this unit's W13 block: KB13 tiles of 64 columns of d
+          const CUtensorMap* m13 = ud.kind == 0 ? &tmW13s : &tmW13;
+          const int row13 = ud.expert * 2 * I + ud.chunk * 128;
+          for (int st = 0; st < KB13 && ok; ++st) ok = load(m13, st * 64, row13);
         }
+        if (ok && prev_kind >= 0) {
+          // the previous unit's W2 rows: MT2 tiles of 128, columns chunk*64 .. +63
+          const CUtensorMap* m2 = prev_kind == 0 ? &tmW2s : &tmW2;
+          for (int m = 0; m < MT2 && ok; ++m)
+            ok = load(m2, prev_chunk * kDecUC, prev_expert * D + m * 128);
+        }
+        if (ud.kind < 0) break;
+        prev_kind = ud.kind;
+        prev_expert = ud.expert;
+        prev_chunk = ud.chunk;
       }
       if (!ok) {
         // a wait ran out: the others see the flag; let the loads in flight land
@@ -431,45 +457,52 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
     if (lane == 0) {
       int q = 0, stage = 0;
       uint32_t qphase = 0, sphase = 0;
-      uint32_t j = 0;
+      uint32_t j = 0;          // units whose gate/up MMAs were issued
       bool ok = true;
+      // unit j's down MMAs follow unit j+1's gate/up MMAs (the ring order)
+      auto down = [&](uint32_t jj) {
+        // the epilogue has read D1 of unit jj and written its a^T
+        if (!wait_bounded(a_ready, jj & 1u, abort_p, a.status)) return false;
+        tc_fence_after();
+        for (int m = 0; m < MT2; ++m) {
+          if (!wait_bounded(full_bar(stage), sphase, abort_p, a.status)) return false;
+          tc_fence_after();
+          const uint32_t sa = ring_base + stage * kDecTileBytes;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16(tmem_base + 2 * kDecN + m * kDecN, desc_kmajor_sw128(sa + k * 32),
+                     desc_kmajor_sw128(at_base + k * 32), IDESC, k > 0 ? 1u : 0u);
+          mma_commit(empty_bar(stage));
+          if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
+        }
+        mma_commit(dn_full);
+        return true;
+      };
       while (ok) {
         if (!wait_bounded(qfull_bar(q), qphase, abort_p, a.status)) { ok = false; break; }
         const int kind = qdesc[q].kind;
         mbar_arrive(qempty_bar(q));
         if (++q == kDecQueue) { q = 0; qphase ^= 1u; }
+        if (kind >= 0) {
+          // gate/up of unit j: D1[j % 2] = W13 block . U^T
+          const uint32_t d1 = tmem_base + (j & 1u) * kDecN;
+          for (int kb = 0; kb < KB13; ++kb) {
+            if (!wait_bounded(full_bar(stage), sphase, abort_p, a.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sa = ring_base + stage * kDecTileBytes;
+            const uint32_t sb = ut_base + kb * (kDecN * 128);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_bf16(d1, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32), IDESC,
+                       (kb > 0 || k > 0) ? 1u : 0u);
+            mma_commit(empty_bar(stage));
+            if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
+          }
+          if (!ok) break;
+          mma_commit(gu_full);
+        }
+        if (j > 0 && !down(j - 1)) { ok = false; break; }
         if (kind < 0) break;
-        // gate/up: D1 = W13 block . U^T
-        for (int kb = 0; kb < KB13; ++kb) {
-          if (!wait_bounded(full_bar(stage), sphase, abort_p, a.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t sa = ring_base + stage * kDecTileBytes;
-          const uint32_t sb = ut_base + kb * (kDecN * 128);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem_base, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32),
-                     IDESC, (kb > 0 || k > 0) ? 1u : 0u);
-          mma_commit(empty_bar(stage));
-          if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
-        }
-        if (!ok) break;
-        mma_commit(gu_full);
-        // down, once the epilogue has read D1 and written a^T
-        if (!wait_bounded(a_ready, j & 1u, abort_p, a.status)) { ok = false; break; }
-        tc_fence_after();
-        for (int m = 0; m < MT2; ++m) {
-          if (!wait_bounded(full_bar(stage), sphase, abort_p, a.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t sa = ring_base + stage * kDecTileBytes;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem_base + kDecN + m * kDecN, desc_kmajor_sw128(sa + k * 32),
-                     desc_kmajor_sw128(at_base + k * 32), IDESC, k > 0 ? 1u : 0u);
-          mma_commit(empty_bar(stage));
-          if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
-        }
-        if (!ok) break;
-        mma_commit(dn_full);
         ++j;
       }
       if (!ok) {
@@ -499,7 +532,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
       if (!epi_all(warp_wait(gu_full, j & 1u, abort_p, a.status))) break;
       tc_fence_after();
       float z[kDecN];
-      tmem_ld16(tl, z);
+      tmem_ld16(tl + (j & 1u) * kDecN, z);
       tmem_ld_wait_regs16(z);
       if (q4 >= 2) {
 #pragma unroll
@@ -523,7 +556,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
       float* base = a.part + static_cast<int64_t>(ud.slot) * D + r;
       for (int m = 0; m < MT2; ++m) {
         float y[kDecN];
-        tmem_ld16(tl + kDecN + m * kDecN, y);
+        tmem_ld16(tl + 2 * kDecN + m * kDecN, y);
         tmem_ld_wait_regs16(y);
 #pragma unroll
         for (int t = 0; t < kDecN; ++t) {
