@@ -15,13 +15,14 @@
 // A unit on the tensor cores (weights as the M = 128 operand, the batch's
 // tokens as N = 16 columns, fp32 accumulators in TMEM):
 //   gate/up  D1[128 x 16] = W13 block [128 x d] . U^T, U = all tokens (bf16,
-//            zero rows past T), in d/64 MMA steps from TMA tiles;
+//            zero rows past T), in d/64 MMA steps; each ring stage brings a
+//            W13 tile and the tokens' tile of the same 64 columns;
 //   SwiGLU   a[r, t] = SiLU(D1[r, t]) * D1[64 + r, t]   (r < 64), bf16;
 //   down     D2[m][128 x 16] = W2[m*128 .. +127, chunk cols] . a, d/128 tiles;
 //   store    the columns of the unit's own tokens (its expert's tokens, or all
 //            of them for a shared expert) as partial rows.
 // Roles (8 warps): warp 0 the TMA producer (unit counter, W13 and W2 tiles into
-// a 9-stage ring, running ahead into the next unit), warp 1 the MMA issuer,
+// an 11-stage ring, running ahead into the next unit), warp 1 the MMA issuer,
 // warp 2 the TMEM owner, warps 4-7 the epilogue (TMEM lane quarters).  The
 // ring carries unit i's W13 tiles before unit i-1's W2 tiles, and D1 is
 // double-buffered, so unit i's gate/up MMAs run while the epilogue turns
@@ -60,7 +61,9 @@ constexpr int kDecThreads = 256;                     // 8 warps
 constexpr int kDecUC = 64;                           // intermediate rows per unit
 constexpr int kDecN = 16;                            // token columns of an MMA
 constexpr int kDecTileBytes = 128 * 64 * 2;          // one 128 x 64 bf16 TMA tile
-constexpr int kDecStages = 9;
+constexpr int kDecUTileBytes = 16 * 64 * 2;          // the tokens' 64 columns (16 rows)
+constexpr int kDecStageBytes = kDecTileBytes + kDecUTileBytes;
+constexpr int kDecStages = 11;
 constexpr int kDecQueue = 4;                         // unit descriptors in flight
 constexpr int kDecRouterExperts = 8;                 // experts per router CTA
 constexpr int kDecMaxSlots = kDecMaxT * 32;          // routed (token, k) slots
@@ -153,7 +156,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
                     const __grid_constant__ CUtensorMap tmW13s,
                     const __grid_constant__ CUtensorMap tmW2,
-                    const __grid_constant__ CUtensorMap tmW2s, const DecArgs a) {
+                    const __grid_constant__ CUtensorMap tmW2s,
+                    const __grid_constant__ CUtensorMap tmU, const DecArgs a) {
   constexpr int D = NV * 256;        // hidden size
   constexpr int KB13 = D / 64;       // gate/up k-blocks per unit
   constexpr int MT2 = D / 128;       // down row tiles per unit
@@ -170,13 +174,12 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
   __shared__ int s_total, s_last;
   __shared__ float upx[64][kDecN + 1];            // the up rows of D1, for the SwiGLU
 
-  // dynamic: ring | U (KB13 tiles of 16 rows) | a^T (one 16-row tile)
+  // dynamic: ring (stage = a weight tile + the tokens' tile of the same k
+  // columns) | a^T (one 16-row tile)
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* ut = ring + kDecStages * kDecTileBytes;
-  uint8_t* at = ut + KB13 * (kDecN * 128);
+  uint8_t* at = ring + kDecStages * kDecStageBytes;
   const uint32_t ring_base = smem_addr(ring);
-  const uint32_t ut_base = smem_addr(ut);
   const uint32_t at_base = smem_addr(at);
   const uint32_t bar_base = smem_addr(bars);
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
@@ -216,15 +219,6 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
   }
   pdl_wait();  // u, the weights and the zeroed sync words come from earlier stream work
   pdl_trigger();
-  // U: every token row as K-major 64-column tiles with 128-byte swizzle,
-  // zero rows past T (the B operand of every gate/up MMA)
-  for (int i = tid; i < kDecN * (D / 8); i += kDecThreads) {
-    const int t = i / (D / 8), c = i - t * (D / 8);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (t < T) v = reinterpret_cast<const uint4*>(a.u + static_cast<int64_t>(t) * D)[c];
-    *reinterpret_cast<uint4*>(ut + (c >> 3) * (kDecN * 128) + sw128_off(t, (c & 7) * 8)) = v;
-  }
-  fence_async_shared();  // generic-proxy writes of U, before the tensor cores read them
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -233,6 +227,10 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
   // ---- 1. router -----------------------------------------------------------
   const int n_rctas = (n + kDecRouterExperts - 1) / kDecRouterExperts;
   if (static_cast<int>(blockIdx.x) < n_rctas) {
+    // the batch's token rows into the (still idle) ring, row-major
+    for (int i = tid; i < T * (D / 8); i += kDecThreads)
+      reinterpret_cast<uint4*>(ring)[i] = reinterpret_cast<const uint4*>(a.u)[i];
+    __syncthreads();
     const int e = blockIdx.x * kDecRouterExperts + warp;
     if (e < n) {
       const uint4* er = reinterpret_cast<const uint4*>(a.E + static_cast<int64_t>(e) * D);
@@ -244,15 +242,10 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
         ev[v][4] = bf_lo(x.z); ev[v][5] = bf_hi(x.z); ev[v][6] = bf_lo(x.w); ev[v][7] = bf_hi(x.w);
       }
       for (int t = 0; t < T; ++t) {
-        // the token's row from the U tiles (16-byte chunk c of row t sits in
-        // tile c / 8 at chunk (c % 8) ^ (t % 8))
+        const uint4* ur = reinterpret_cast<const uint4*>(ring + t * D * 2);
         uint4 uv[NV];
 #pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          const int c = v * 32 + lane;
-          uv[v] = *reinterpret_cast<const uint4*>(ut + (c >> 3) * (kDecN * 128) +
-                                                  sw128_off(t, (c & 7) * 8));
-        }
+        for (int v = 0; v < NV; ++v) uv[v] = ur[v * 32 + lane];
         float acc = 0.0f;
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
@@ -348,6 +341,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
     if (lane == 0) {
       tma_prefetch_desc(&tmW13);
       tma_prefetch_desc(&tmW2);
+      tma_prefetch_desc(&tmU);
       if (Ks > 0) {
         tma_prefetch_desc(&tmW13s);
         tma_prefetch_desc(&tmW2s);
@@ -414,11 +408,14 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
         if (++q == kDecQueue) { q = 0; qphase ^= 1u; }
         // the ring order is W13(unit i), then W2(unit i-1): the MMAs of unit
         // i's gate/up run while the epilogue turns unit i-1's into a^T
-        auto load = [&](const CUtensorMap* map, int x, int y) {
+        // with_u: also the tokens' tile of the same 64 columns of d (rows past
+        // T read as zeros), the B operand of the gate/up MMAs
+        auto load = [&](const CUtensorMap* map, int x, int y, bool with_u) {
           if (!wait_bounded(empty_bar(stage), sphase ^ 1u, abort_p, a.status)) return false;
-          const uint32_t dst = ring_base + stage * kDecTileBytes;
-          mbar_arrive_expect_tx(full_bar(stage), kDecTileBytes);
+          const uint32_t dst = ring_base + stage * kDecStageBytes;
+          mbar_arrive_expect_tx(full_bar(stage), kDecTileBytes + (with_u ? kDecUTileBytes : 0));
           tma_load_2d(dst, map, full_bar(stage), x, y);
+          if (with_u) tma_load_2d(dst + kDecTileBytes, &tmU, full_bar(stage), x, 0);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (sphase << stage);
           if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
@@ -428,13 +425,13 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
           // this unit's W13 block: KB13 tiles of 64 columns of d
           const CUtensorMap* m13 = ud.kind == 0 ? &tmW13s : &tmW13;
           const int row13 = ud.expert * 2 * I + ud.chunk * 128;
-          for (int st = 0; st < KB13 && ok; ++st) ok = load(m13, st * 64, row13);
+          for (int st = 0; st < KB13 && ok; ++st) ok = load(m13, st * 64, row13, true);
         }
         if (ok && prev_kind >= 0) {
           // the previous unit's W2 rows: MT2 tiles of 128, columns chunk*64 .. +63
           const CUtensorMap* m2 = prev_kind == 0 ? &tmW2s : &tmW2;
           for (int m = 0; m < MT2 && ok; ++m)
-            ok = load(m2, prev_chunk * kDecUC, prev_expert * D + m * 128);
+            ok = load(m2, prev_chunk * kDecUC, prev_expert * D + m * 128, false);
         }
         if (ud.kind < 0) break;
         prev_kind = ud.kind;
@@ -467,7 +464,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
         for (int m = 0; m < MT2; ++m) {
           if (!wait_bounded(full_bar(stage), sphase, abort_p, a.status)) return false;
           tc_fence_after();
-          const uint32_t sa = ring_base + stage * kDecTileBytes;
+          const uint32_t sa = ring_base + stage * kDecStageBytes;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_bf16(tmem_base + 2 * kDecN + m * kDecN, desc_kmajor_sw128(sa + k * 32),
@@ -489,8 +486,8 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
           for (int kb = 0; kb < KB13; ++kb) {
             if (!wait_bounded(full_bar(stage), sphase, abort_p, a.status)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sa = ring_base + stage * kDecTileBytes;
-            const uint32_t sb = ut_base + kb * (kDecN * 128);
+            const uint32_t sa = ring_base + stage * kDecStageBytes;
+            const uint32_t sb = sa + kDecTileBytes;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               mma_bf16(d1, desc_kmajor_sw128(sa + k * 32), desc_kmajor_sw128(sb + k * 32), IDESC,
@@ -637,18 +634,17 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
   }
 }
 
-constexpr int dec_smem_bytes(int D) {
-  return 1024 + kDecStages * kDecTileBytes + (D / 64) * kDecN * 128 + kDecN * 128;
-}
+constexpr int dec_smem_bytes(int) { return 1024 + kDecStages * kDecStageBytes + kDecN * 128; }
 
 template <int NV>
 int launch_decode_nv(const CUtensorMap& m13, const CUtensorMap& m13s, const CUtensorMap& m2,
-                     const CUtensorMap& m2s, const DecArgs& a, int grid, cudaStream_t st) {
+                     const CUtensorMap& m2s, const CUtensorMap& mu, const DecArgs& a, int grid,
+                     cudaStream_t st) {
   static std::atomic<uint64_t> optin{0};
   auto kern = decode_layer_kernel<NV>;
   const int smem = dec_smem_bytes(NV * 256);
   if (int rc = ensure_smem_optin(reinterpret_cast<const void*>(kern), smem, optin)) return rc;
-  return launch_k(kern, grid, kDecThreads, smem, st, 1, m13, m13s, m2, m2s, a);
+  return launch_k(kern, grid, kDecThreads, smem, st, 1, m13, m13s, m2, m2s, mu, a);
 }
 
 }  // namespace
@@ -686,6 +682,11 @@ int launch_decode_fused(const moe_shape_t& s, const void* u, const void* E, cons
     m13s = m13;
     m2s = m2;
   }
+  // the tokens as 16-row boxes of 64 columns (rows past T read as zeros)
+  CUtensorMap mu;
+  if (!make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u, d, static_cast<uint64_t>(s.T), d * 2,
+                   64, kDecN))
+    return MOE_ERR_CUDA;
   if (cudaMemsetAsync(sync, 0, sizeof(DecSync), st) != cudaSuccess) return MOE_ERR_CUDA;
   DecArgs a{};
   a.u = static_cast<const bf16*>(u);
@@ -706,10 +707,10 @@ int launch_decode_fused(const moe_shape_t& s, const void* u, const void* E, cons
   a.K = s.top_k;
   a.flags = s.flags;
   switch (s.d) {
-    case 256: return launch_decode_nv<1>(m13, m13s, m2, m2s, a, sms, st);
-    case 512: return launch_decode_nv<2>(m13, m13s, m2, m2s, a, sms, st);
-    case 1024: return launch_decode_nv<4>(m13, m13s, m2, m2s, a, sms, st);
-    case 2048: return launch_decode_nv<8>(m13, m13s, m2, m2s, a, sms, st);
+    case 256: return launch_decode_nv<1>(m13, m13s, m2, m2s, mu, a, sms, st);
+    case 512: return launch_decode_nv<2>(m13, m13s, m2, m2s, mu, a, sms, st);
+    case 1024: return launch_decode_nv<4>(m13, m13s, m2, m2s, mu, a, sms, st);
+    case 2048: return launch_decode_nv<8>(m13, m13s, m2, m2s, mu, a, sms, st);
     default: return MOE_ERR_SHAPE;
   }
 }

@@ -28,16 +28,7 @@ namespace {
 constexpr int PBM = 256;   // rows per pair tile
 constexpr int HBM_ROWS = 128;  // rows per CTA
 constexpr int PBK = 64;
-// Epilogue warps: two per TMEM lane quarter, each draining half of the
-// columns.  Four (one per quarter, every column) leave four staging areas of
-// shared memory to the operand ring, six 32 KB stages for 256-column tiles
-// and four 48 KB stages for 512-column tiles against five and three; that
-// measured no faster for 256-column tiles (76.9% against 76.7% tensor-pipe
-// busy on the 16B-shaped gate/up GEMM) and slower for 512-column tiles,
-// whose single accumulator waits for the epilogue (66.3% against 72.6% on
-// the 16B-shaped down GEMM).
-constexpr int kPairEpiWarps = 8;
-constexpr int kPairThreads = 128 + 32 * kPairEpiWarps;  // 4 role warps + the epilogue
+constexpr int kPairThreads = 384;  // 4 role warps + 8 epilogue warps
 constexpr int kPairMaxGroups = 257;
 
 // Epilogue staging: every epilogue warp owns 32 rows x (128 + 16) bytes of
@@ -47,7 +38,7 @@ constexpr int kStageRowBytes = 128;
 constexpr int kStagePitch = kStageRowBytes + 16;
 constexpr int kWarpStageBytes = 32 * kStagePitch;
 
-template <int EPI> constexpr int pair_epi_warps() { return kPairEpiWarps; }
+template <int EPI> constexpr int pair_epi_warps() { return 8; }
 
 // pipeline depth: as many 256-row k-block stages as fit beside the staging
 template <int BN, int EPI>
@@ -311,7 +302,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
   } else if (warp >= 4 && warp < 4 + EPI_WARPS) {
     // ------------------------------------------------------- epilogue -----
     const int q = warp & 3;          // TMEM lane quarter of this warp
-    constexpr int HCOLS = 8 / EPI_WARPS;  // halves of the tile's columns a warp drains
+    const int hcol = (warp - 4) >> 2;  // which half of the tile's columns it drains
     const int r = q * 32 + lane;
     const uint32_t tempty_leader0 = map_to_cta(tempty_bar(0), 0);
     const uint32_t tempty_leader1 = map_to_cta(tempty_bar(1), 0);
@@ -335,9 +326,6 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
       uint8_t* stage = smem + STAGES * STAGE_BYTES + (warp - 4) * kWarpStageBytes;
-#pragma unroll 1
-      for (int hh = 0; hh < HCOLS; ++hh) {
-      const int hcol = HCOLS == 1 ? (warp - 4) >> 2 : hh;
       if (EPI == kEpiSwiGLU) {
         // this warp's output columns: 64 (BN = 256) or 32 (BN = 128)
         constexpr int OC = BN / 4;
@@ -423,7 +411,6 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
           }
         }
       }
-      }  // column halves
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
@@ -451,7 +438,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r,
 // ---------------------------------------------------------------------------
 constexpr int kWideBN = 512;
 constexpr int kWideHalf = 256;
-constexpr int kWideEpiWarps = kPairEpiWarps;
+constexpr int kWideEpiWarps = 8;
 
 // Stage size and count by the k-block width BKW (kWideBK): 64 gives three
 // 48 KB stages beside the epilogue staging.
@@ -636,75 +623,39 @@ grouped_gemm_pair_wide_kernel(const __grid_constant__ CUtensorMap tmA_r,
   } else if (warp == 1) {
     // ----------------------------------------- MMA issuer (leader only) ----
     if (lane == 0 && leader) {
-      // Stages are consumed in order.  At the start of a tile the half-1
-      // accumulator may still be draining: the half-0 MMAs of the first
-      // k-blocks run ahead (their stages stay held) until half 1 is free or
-      // every stage is held, then half 1 catches up and the two run in step.
-      int st0 = 0, st1 = 0;      // next stage to wait for / to release
-      uint32_t ph0 = 0;
+      int stage = 0;
+      uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      auto mma_half = [&](int st, int h, int kb) {
-        const uint32_t sa = smem_base + st * STAGE_BYTES;
-        const uint32_t sb = sa + A_BYTES;
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(h * kWideHalf);
-#pragma unroll
-        for (int k = 0; k < BKW / 16; ++k) {
-          mma_bf16_pair(d_tmem, wide_desc<BKW>(sa + k * 32),
-                        wide_desc<BKW>(sb + h * BH_BYTES + k * 32), IDESC,
-                        (kb > 0 || k > 0) ? 1u : 0u);
-        }
-      };
       for (int tile = cluster; tile < total_tiles && ok; tile += nclusters, ++it) {
         const PairTile ti =
             decode_pair_tile(place_tile(tile, total_tiles, nclusters, n_long), tile_start, G, hs,
                              args.nt_routed, args.nt_shared);
         const int nkb = ti.shared ? args.kb_shared : args.kb_routed;
         const uint32_t tp = static_cast<uint32_t>(it & 1);
-        // the epilogue has drained half 0 of the previous tile
-        if (!wait_bounded(tempty_bar(0), tp ^ 1u, abort_p, args.status)) { ok = false; break; }
-        tc_fence_after();
-        bool free1 = false;
-        int kb1 = 0;  // next k-block whose half-1 MMAs are due
-        for (int kb0 = 0; kb0 < nkb && ok; ++kb0) {
-          if (!free1 && kb0 - kb1 == STAGES) {
-            // every stage holds a k-block still due for half 1: wait for it
-            if (!wait_bounded(tempty_bar(1), tp ^ 1u, abort_p, args.status)) { ok = false; break; }
-            tc_fence_after();
-            free1 = true;
-            for (; kb1 < kb0; ++kb1) {
-              mma_half(st1, 1, kb1);
-              mma_commit_pair(empty_bar(st1), kBoth);
-              if (++st1 == STAGES) st1 = 0;
-            }
-          }
-          if (!wait_bounded(full_bar(st0), ph0, abort_p, args.status)) { ok = false; break; }
+        for (int kb = 0; kb < nkb && ok; ++kb) {
+          if (!wait_bounded(full_bar(stage), phase, abort_p, args.status)) { ok = false; break; }
           tc_fence_after();
-          mma_half(st0, 0, kb0);
-          if (kb0 == nkb - 1) mma_commit_pair(tfull_bar(0), kBoth);
-          if (++st0 == STAGES) { st0 = 0; ph0 ^= 1u; }
-          if (!free1 && mbar_try_wait(tempty_bar(1), tp ^ 1u)) {
-            tc_fence_after();
-            free1 = true;
-          }
-          if (free1) {
-            for (; kb1 <= kb0; ++kb1) {
-              mma_half(st1, 1, kb1);
-              if (kb1 == nkb - 1) mma_commit_pair(tfull_bar(1), kBoth);
-              mma_commit_pair(empty_bar(st1), kBoth);
-              if (++st1 == STAGES) st1 = 0;
+          const uint32_t sa = smem_base + stage * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+          for (int h = 0; h < 2; ++h) {
+            if (kb == 0) {
+              // the epilogue has drained this half of the previous tile
+              if (!wait_bounded(tempty_bar(h), tp ^ 1u, abort_p, args.status)) { ok = false; break; }
+              tc_fence_after();
             }
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(h * kWideHalf);
+#pragma unroll
+            for (int k = 0; k < BKW / 16; ++k) {
+              mma_bf16_pair(d_tmem, wide_desc<BKW>(sa + k * 32),
+                            wide_desc<BKW>(sb + h * BH_BYTES + k * 32), IDESC,
+                            (kb > 0 || k > 0) ? 1u : 0u);
+            }
+            if (kb == nkb - 1) mma_commit_pair(tfull_bar(h), kBoth);
           }
-        }
-        if (ok && !free1) {
-          if (!wait_bounded(tempty_bar(1), tp ^ 1u, abort_p, args.status)) { ok = false; break; }
-          tc_fence_after();
-          for (; kb1 < nkb; ++kb1) {
-            mma_half(st1, 1, kb1);
-            if (kb1 == nkb - 1) mma_commit_pair(tfull_bar(1), kBoth);
-            mma_commit_pair(empty_bar(st1), kBoth);
-            if (++st1 == STAGES) st1 = 0;
-          }
+          if (!ok) break;
+          mma_commit_pair(empty_bar(stage), kBoth);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       if (!ok) {
@@ -718,7 +669,7 @@ grouped_gemm_pair_wide_kernel(const __grid_constant__ CUtensorMap tmA_r,
   } else if (warp >= 4 && warp < 4 + EPI_WARPS) {
     // ------------------------------------------------------- epilogue -----
     const int q = warp & 3;             // TMEM lane quarter of this warp
-    constexpr int HC = 8 / EPI_WARPS;   // 128-column parts of a half a warp drains
+    const int hc = (warp - 4) >> 2;     // which 128 columns of a half it drains
     const int r = q * 32 + lane;
     const uint32_t tempty_leader0 = map_to_cta(tempty_bar(0), 0);
     const uint32_t tempty_leader1 = map_to_cta(tempty_bar(1), 0);
@@ -741,9 +692,6 @@ grouped_gemm_pair_wide_kernel(const __grid_constant__ CUtensorMap tmA_r,
       for (int h = 0; h < 2; ++h) {
         if (!wait_bounded(tfull_bar(h), tp, abort_p, args.status)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll 1
-        for (int pp = 0; pp < HC; ++pp) {
-        const int hc = HC == 1 ? (warp - 4) >> 2 : pp;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                static_cast<uint32_t>(h * kWideHalf + hc * 128);
         if (EPI == kEpiSwiGLU) {
@@ -816,7 +764,6 @@ grouped_gemm_pair_wide_kernel(const __grid_constant__ CUtensorMap tmA_r,
             }
           }
         }
-        }  // 128-column parts
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(h ? tempty_leader1 : tempty_leader0);
