@@ -29,18 +29,27 @@
 // unit i-1's D1 into a^T.
 //
 // Phases, all in this one launch (one CTA per SM):
-//  1. Router (CTAs 0 .. ceil(n/8)-1): logits u_t . e_i for 8 experts each,
-//     all tokens, fp32 FMA chains per lane plus a fixed shuffle tree; the CTA
-//     that finishes last runs softmax and top-K for every token (lower expert
-//     index first on ties, gates not renormalised) and publishes idx / w.
-//  2. Units: the shared experts' units need no routing and come first; the
+//  1. Logits (with G = min(n, grid), CTA c < G takes experts c, c + G, ...): expert
+//     i's row stays in registers while each warp takes two tokens,
+//     u_t . e_i as fp32 FMA chains per lane plus a fixed shuffle tree; the
+//     CTA publishes its logits and counts itself.
+//  2. Routing and tables (warps 2-7 of every CTA, the same arithmetic in
+//     each): once every logit CTA is counted, softmax of each token over the
+//     routed experts (fixed-order max and sum) and its top K by rank among
+//     the keys (larger first, lower index first on ties; gates not
+//     renormalised); then each slot's rank within its expert in slot order
+//     (warp match / popc, 32 slots at a time), the experts' offsets and the
+//     active list from warp scans; the producer is released through an
+//     mbarrier.
+//  3. Units: the shared experts' units need no routing and come first; the
 //     routed units (active experts in increasing index, chunks in order)
-//     become known once the routing is published.
-//  3. Combine: once every unit is done, h_t = u_t + sum_j g_j p_j over the
+//     wait for the tables.
+//  4. Combine: once every unit is done, h_t = u_t + sum_j g_j p_j over the
 //     token's partial rows p_j (the shared units' with g = 1, then each
-//     routed slot k's chunks with g = w[t,k]), in fp32: one warp per (token,
-//     4 columns), lane l summing rows l, l + 32, ... in order, then a fixed
-//     shuffle tree; u is added last and h rounded once to bf16.
+//     routed slot k's chunks with g = w[t,k]), in fp32: one CTA per (token,
+//     256 columns), warp w summing rows w, w + 8, ... in order (coalesced
+//     row segments, 8 rows' loads in flight), then the 8 warps' sums in warp
+//     order; u is added last and h rounded once to bf16.
 // Every wait is bounded: a wait that runs out records MOE_ERR_DEVICE_CHECK in
 // the status word and the kernel winds down without writing h.
 #include <cuda.h>
@@ -65,17 +74,17 @@ constexpr int kDecUTileBytes = 16 * 64 * 2;          // the tokens' 64 columns (
 constexpr int kDecStageBytes = kDecTileBytes + kDecUTileBytes;
 constexpr int kDecStages = 11;
 constexpr int kDecQueue = 4;                         // unit descriptors in flight
-constexpr int kDecRouterExperts = 8;                 // experts per router CTA
+constexpr int kRouteWarps = 6;                       // warps 2-7 route the tokens
 constexpr int kDecMaxSlots = kDecMaxT * 32;          // routed (token, k) slots
 constexpr uint32_t kDecTmemCols = 512;               // D1 (2 x 16) + D2 (16 per 128 rows of d)
 static_assert(kDecMaxT <= kDecN, "the batch fits one MMA's columns");
 
 // sync words of the decode scratch (zeroed before each launch)
 struct DecSync {
-  int unit_next;     // next unit to take
-  int route_arrive;  // router CTAs done with their logits
-  int route_done;    // 1 once idx / w are published
-  int units_done;    // units whose partials are written
+  int unit_next;      // next unit to take
+  int logit_ctas;     // CTAs whose logits are published
+  int units_done;     // units whose partials are written
+  int pad;
 };
 
 struct DecArgs {
@@ -120,6 +129,21 @@ __device__ __forceinline__ bool epi_all(bool v) {
   return r != 0;
 }
 
+// The routing warps 2-7 vote (named barrier 2): true when all 192 threads
+// pass true.
+__device__ __forceinline__ bool route_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 2, 192, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+
 // a bounded mbarrier wait taken by a whole warp, with one result for it
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           int32_t* status) {
@@ -145,6 +169,86 @@ __device__ __forceinline__ bool spin_until(const int* p, int target, int32_t* st
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
+// Softmax and top-K of tokens t0, t0 + tstep, ... < T, one warp; lane l holds
+// experts l, l + 32, ..., l + 32 (NQ - 1) (NQ * 32 >= n).  keys: this warp's
+// shared row of 4 * ceil(n / 4) floats.  Each selected expert e of token t
+// goes to slot rank(e), its rank among the keys (larger first, lower index
+// first on ties); gates are exp(l_e - max) / sum, not renormalised.
+template <int NQ>
+__device__ __forceinline__ void route_tokens(const float* logits, const float* bias, int n, int K,
+                                             int T, int t0, int tstep, bool select_only,
+                                             float* keys, int* sidx, float* sw, int32_t* gidx,
+                                             float* gw) {
+  const int lane = threadIdx.x & 31;
+  const int n4 = (n + 3) & ~3;
+  float b[NQ], nxt[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int e = lane + 32 * q;
+    b[q] = (bias && e < n) ? bias[e] : 0.0f;
+    nxt[q] = (t0 < T && e < n) ? __ldcg(logits + t0 * n + e) : 0.0f;
+  }
+#pragma unroll 1
+  for (int t = t0; t < T; t += tstep) {
+    float key[NQ], lg[NQ];
+    float m = -CUDART_INF_F;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int e = lane + 32 * q;
+      const float raw = nxt[q];
+      nxt[q] = (t + tstep < T && e < n) ? __ldcg(logits + (t + tstep) * n + e) : 0.0f;
+      key[q] = e < n ? raw + b[q] : -CUDART_INF_F;
+      lg[q] = e < n ? (select_only ? raw : key[q]) : -CUDART_INF_F;
+      if (e < n4) keys[e] = key[q];
+      m = fmaxf(m, lg[q]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float ex[NQ], z = 0.0f;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      ex[q] = lane + 32 * q < n ? expf(lg[q] - m) : 0.0f;
+      z += ex[q];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    const float inv_z = 1.0f / z;
+    __syncwarp();
+    int rank[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) rank[q] = 0;
+    const float4* k4 = reinterpret_cast<const float4*>(keys);
+#pragma unroll 2
+    for (int j4 = 0; j4 < n4 / 4; ++j4) {
+      const float4 v = k4[j4];
+      const int j = 4 * j4;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int e = lane + 32 * q;
+        const float kq = key[q];
+        rank[q] += static_cast<int>(v.x > kq) | (static_cast<int>(v.x == kq) & static_cast<int>(j < e));
+        rank[q] += static_cast<int>(v.y > kq) | (static_cast<int>(v.y == kq) & static_cast<int>(j + 1 < e));
+        rank[q] += static_cast<int>(v.z > kq) | (static_cast<int>(v.z == kq) & static_cast<int>(j + 2 < e));
+        rank[q] += static_cast<int>(v.w > kq) | (static_cast<int>(v.w == kq) & static_cast<int>(j + 3 < e));
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int e = lane + 32 * q;
+      if (e < n && rank[q] < K) {
+        const float g = ex[q] * inv_z;
+        sidx[t * K + rank[q]] = e;
+        sw[t * K + rank[q]] = g;
+        if (gidx) {
+          gidx[t * K + rank[q]] = e;
+          gw[t * K + rank[q]] = g;
+        }
+      }
+    }
+    __syncwarp();  // keys[] is rewritten for the next token
+  }
+}
+
 // byte offset of element (row, k) in a K-major [rows x 64] bf16 tile with
 // 128-byte swizzle (16-byte chunk k/8 of a row sits at chunk (k/8) ^ (row % 8))
 __device__ __forceinline__ uint32_t sw128_off(int row, int k) {
@@ -163,7 +267,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
   constexpr int MT2 = D / 128;       // down row tiles per unit
   constexpr uint32_t IDESC = idesc_bf16_f32(128, kDecN);
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[2 * kDecStages + 2 * kDecQueue + 4];
+  __shared__ __align__(8) uint64_t bars[2 * kDecStages + 2 * kDecQueue + 6];
   __shared__ UnitDesc qdesc[kDecQueue];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -171,6 +275,8 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
   __shared__ int s_tok[kDecMaxSlots];             // tokens of each expert, increasing t
   __shared__ int s_rank[kDecMaxSlots];            // rank of token t within expert idx[t,k]
   __shared__ int s_idx[kDecMaxSlots];
+  __shared__ float s_w[kDecMaxSlots];             // gates of the slots
+  __shared__ __align__(16) float s_keys[kRouteWarps][256];  // each routing warp's token keys
   __shared__ int s_total, s_last;
   __shared__ float upx[64][kDecN + 1];            // the up rows of D1, for the SwiGLU
 
@@ -186,10 +292,15 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
   auto empty_bar = [&](int s) { return bar_base + 8u * (kDecStages + s); };
   auto qfull_bar = [&](int q) { return bar_base + 8u * (2 * kDecStages + q); };
   auto qempty_bar = [&](int q) { return bar_base + 8u * (2 * kDecStages + kDecQueue + q); };
-  const uint32_t gu_full = bar_base + 8u * (2 * kDecStages + 2 * kDecQueue);
-  const uint32_t a_ready = gu_full + 8u;
-  const uint32_t dn_full = gu_full + 16u;
-  const uint32_t drain_bar = gu_full + 24u;
+  // gate/up done, one barrier per D1 buffer: the MMA thread commits unit
+  // j + 1's gate/up before it waits for unit j's a^T, so a single barrier
+  // could complete two phases before the epilogue tests unit j's parity
+  const uint32_t gu_full0 = bar_base + 8u * (2 * kDecStages + 2 * kDecQueue);
+  auto gu_full = [&](uint32_t j) { return gu_full0 + 8u * (j & 1u); };
+  const uint32_t a_ready = gu_full0 + 16u;
+  const uint32_t dn_full = gu_full0 + 24u;
+  const uint32_t drain_bar = gu_full0 + 32u;
+  const uint32_t tables_bar = gu_full0 + 40u;  // warp 3's expert tables are built
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = a.T, n = a.n, K = a.K, I = a.I, Ks = a.Ks;
@@ -206,12 +317,15 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
       mbar_init(qfull_bar(q), 1);
       mbar_init(qempty_bar(q), 5);  // the MMA thread and the 4 epilogue warps
     }
-    mbar_init(gu_full, 1);
+    mbar_init(gu_full(0), 1);
+    mbar_init(gu_full(1), 1);
     mbar_init(a_ready, 1);
     mbar_init(dn_full, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(tables_bar, 32);
     abort_flag = 0;
     fence_mbar_init();
+    fence_async_shared();  // the initialised barriers, before TMA completes on them
   }
   if (warp == 2) {
     tmem_alloc(smem_addr(&tmem_slot), kDecTmemCols);
@@ -224,115 +338,48 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
 
-  // ---- 1. router -----------------------------------------------------------
-  const int n_rctas = (n + kDecRouterExperts - 1) / kDecRouterExperts;
-  if (static_cast<int>(blockIdx.x) < n_rctas) {
-    // the batch's token rows into the (still idle) ring, row-major
-    for (int i = tid; i < T * (D / 8); i += kDecThreads)
-      reinterpret_cast<uint4*>(ring)[i] = reinterpret_cast<const uint4*>(a.u)[i];
-    __syncthreads();
-    const int e = blockIdx.x * kDecRouterExperts + warp;
-    if (e < n) {
+  // ---- 1. logits: CTA c takes experts c, c + n_lc, ... ---------------------
+  const int n_lc = n < static_cast<int>(gridDim.x) ? n : static_cast<int>(gridDim.x);
+  if (static_cast<int>(blockIdx.x) < n_lc) {
+    const int t0 = warp, t1 = warp + kDecThreads / 32;  // T <= 16: two tokens per warp
+    for (int e = blockIdx.x; e < n; e += n_lc) {
       const uint4* er = reinterpret_cast<const uint4*>(a.E + static_cast<int64_t>(e) * D);
-      float ev[NV][8];
+      const uint4* u0 = reinterpret_cast<const uint4*>(a.u + static_cast<int64_t>(t0 < T ? t0 : 0) * D);
+      const uint4* u1 = reinterpret_cast<const uint4*>(a.u + static_cast<int64_t>(t1 < T ? t1 : 0) * D);
+      uint4 ev[NV], x0[NV], x1[NV];
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        const uint4 x = er[v * 32 + lane];
-        ev[v][0] = bf_lo(x.x); ev[v][1] = bf_hi(x.x); ev[v][2] = bf_lo(x.y); ev[v][3] = bf_hi(x.y);
-        ev[v][4] = bf_lo(x.z); ev[v][5] = bf_hi(x.z); ev[v][6] = bf_lo(x.w); ev[v][7] = bf_hi(x.w);
+        ev[v] = __ldg(er + v * 32 + lane);
+        x0[v] = __ldg(u0 + v * 32 + lane);
+        x1[v] = __ldg(u1 + v * 32 + lane);
       }
-      for (int t = 0; t < T; ++t) {
-        const uint4* ur = reinterpret_cast<const uint4*>(ring + t * D * 2);
-        uint4 uv[NV];
+      float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
-        for (int v = 0; v < NV; ++v) uv[v] = ur[v * 32 + lane];
-        float acc = 0.0f;
+      for (int v = 0; v < NV; ++v) {
+        const uint4 y = ev[v], p = x0[v], q = x1[v];
+        acc0 = fmaf(bf_lo(p.x), bf_lo(y.x), acc0); acc0 = fmaf(bf_hi(p.x), bf_hi(y.x), acc0);
+        acc0 = fmaf(bf_lo(p.y), bf_lo(y.y), acc0); acc0 = fmaf(bf_hi(p.y), bf_hi(y.y), acc0);
+        acc0 = fmaf(bf_lo(p.z), bf_lo(y.z), acc0); acc0 = fmaf(bf_hi(p.z), bf_hi(y.z), acc0);
+        acc0 = fmaf(bf_lo(p.w), bf_lo(y.w), acc0); acc0 = fmaf(bf_hi(p.w), bf_hi(y.w), acc0);
+        acc1 = fmaf(bf_lo(q.x), bf_lo(y.x), acc1); acc1 = fmaf(bf_hi(q.x), bf_hi(y.x), acc1);
+        acc1 = fmaf(bf_lo(q.y), bf_lo(y.y), acc1); acc1 = fmaf(bf_hi(q.y), bf_hi(y.y), acc1);
+        acc1 = fmaf(bf_lo(q.z), bf_lo(y.z), acc1); acc1 = fmaf(bf_hi(q.z), bf_hi(y.z), acc1);
+        acc1 = fmaf(bf_lo(q.w), bf_lo(y.w), acc1); acc1 = fmaf(bf_hi(q.w), bf_hi(y.w), acc1);
+      }
 #pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          acc = fmaf(bf_lo(uv[v].x), ev[v][0], acc); acc = fmaf(bf_hi(uv[v].x), ev[v][1], acc);
-          acc = fmaf(bf_lo(uv[v].y), ev[v][2], acc); acc = fmaf(bf_hi(uv[v].y), ev[v][3], acc);
-          acc = fmaf(bf_lo(uv[v].z), ev[v][4], acc); acc = fmaf(bf_hi(uv[v].z), ev[v][5], acc);
-          acc = fmaf(bf_lo(uv[v].w), ev[v][6], acc); acc = fmaf(bf_hi(uv[v].w), ev[v][7], acc);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) a.logits[t * n + e] = acc;
+      for (int o = 16; o > 0; o >>= 1) {
+        acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
+        acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+      }
+      if (lane == 0) {
+        if (t0 < T) a.logits[t0 * n + e] = acc0;
+        if (t1 < T) a.logits[t1 * n + e] = acc1;
       }
     }
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&a.sync->route_arrive, 1) == n_rctas - 1;
-    __syncthreads();
-    if (s_last) {
-      // the last router CTA: softmax and top-K of every token, warp per token
-      __threadfence();
-      const bool select_only = (a.flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
-      for (int t = warp; t < T; t += kDecThreads / 32) {
-        float lg[8], key[8], ex[8];
-        float m = -CUDART_INF_F;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int ee = lane + 32 * q;
-          float l = -CUDART_INF_F, kv = -CUDART_INF_F;
-          if (ee < n) {
-            const float raw = __ldcg(a.logits + t * n + ee);
-            kv = raw + (a.bias ? a.bias[ee] : 0.0f);
-            l = select_only ? raw : kv;
-          }
-          lg[q] = l;
-          key[q] = kv;
-          m = fmaxf(m, l);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float z = 0.0f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          ex[q] = (lane + 32 * q < n) ? expf(lg[q] - m) : 0.0f;
-          z += ex[q];
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-        const float inv_z = 1.0f / z;
-        unsigned taken = 0;
-        for (int k = 0; k < K; ++k) {
-          float bv = -CUDART_INF_F;
-          int bi = 0x7fffffff;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int ee = lane + 32 * q;
-            if (!((taken >> q) & 1u) && ee < n && (key[q] > bv || bi == 0x7fffffff)) {
-              bv = key[q];
-              bi = ee;
-            }
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) {
-              bv = ov;
-              bi = oi;
-            }
-          }
-          if ((bi & 31) == lane) {
-            taken |= 1u << (bi >> 5);
-            float g = 0.0f;
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              if (q == (bi >> 5)) g = ex[q];
-            a.idx[t * K + k] = bi;
-            a.w[t * K + k] = g * inv_z;
-          }
-        }
-      }
-      __threadfence();
-      __syncthreads();
-      if (tid == 0) {
-        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(&a.sync->route_done), "r"(1)
-                     : "memory");
-      }
-    }
+    if (tid == 0)
+      asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(&a.sync->logit_ctas) : "memory");
   }
 
   // ---- 2. units --------------------------------------------------------------
@@ -354,31 +401,11 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
       while (ok) {
         const int u = atomicAdd(&a.sync->unit_next, 1);
         if (u >= S && !have_tables) {
-          // the routed units need the routing: build the expert tables
-          if (!spin_until(&a.sync->route_done, 1, a.status)) { ok = false; break; }
-          for (int e = 0; e < n; ++e) s_cnt[e] = 0;
-          // idx in batches of 16 independent loads, then the counting sort
-          for (int i0 = 0; i0 < T * K; i0 += 16) {
-            int v[16];
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) v[jj] = i0 + jj < T * K ? __ldcg(a.idx + i0 + jj) : 0;
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj)
-              if (i0 + jj < T * K) s_idx[i0 + jj] = v[jj];
+          // the routed units need the expert tables (warp 3)
+          if (!wait_bounded(tables_bar, 0, abort_p, a.status)) {
+            ok = false;
+            break;
           }
-          for (int i = 0; i < T * K; ++i) {
-            const int e = s_idx[i];
-            s_rank[i] = s_cnt[e]++;  // i runs in increasing t: ranks follow t
-          }
-          int run = 0, na = 0;
-          for (int e = 0; e < n; ++e) {
-            s_off[e] = run;
-            run += s_cnt[e];
-            if (s_cnt[e] > 0) s_active[na++] = e;
-          }
-          s_off[n] = run;
-          for (int i = 0; i < T * K; ++i) s_tok[s_off[s_idx[i]] + s_rank[i]] = i / K;
-          s_total = S + na * nc;
           have_tables = true;
         }
         UnitDesc ud;
@@ -496,7 +523,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
             if (++stage == kDecStages) { stage = 0; sphase ^= 1u; }
           }
           if (!ok) break;
-          mma_commit(gu_full);
+          mma_commit(gu_full(j));
         }
         if (j > 0 && !down(j - 1)) { ok = false; break; }
         if (kind < 0) break;
@@ -511,7 +538,94 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else {
+    // ---------------------------------- routing (warps 2-7) and tables (3) ----
+    // the epilogue warps route too: their first wait (a unit's gate/up) is
+    // further away than the routing
+    const int pw = warp - 2;  // tokens pw, pw + 6, ...
+    bool ok = true;
+    if (tid == 64) ok = spin_until(&a.sync->logit_ctas, n_lc, a.status);
+    ok = route_all(ok);  // warps 2-7 learn the outcome together
+    if (!ok) {
+      if (lane == 0) *abort_p = 1;
+    } else {
+      const bool select_only = (a.flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
+      int32_t* gidx = blockIdx.x == 0 ? a.idx : nullptr;  // one copy of idx / w in the workspace
+      float* gw = blockIdx.x == 0 ? a.w : nullptr;
+      if (n <= 32)
+        route_tokens<1>(a.logits, a.bias, n, K, T, pw, kRouteWarps, select_only, s_keys[pw], s_idx, s_w,
+                        gidx, gw);
+      else if (n <= 64)
+        route_tokens<2>(a.logits, a.bias, n, K, T, pw, kRouteWarps, select_only, s_keys[pw], s_idx, s_w,
+                        gidx, gw);
+      else if (n <= 128)
+        route_tokens<4>(a.logits, a.bias, n, K, T, pw, kRouteWarps, select_only, s_keys[pw], s_idx, s_w,
+                        gidx, gw);
+      else
+        route_tokens<8>(a.logits, a.bias, n, K, T, pw, kRouteWarps, select_only, s_keys[pw], s_idx, s_w,
+                        gidx, gw);
+      asm volatile("bar.sync 2, 192;" ::: "memory");  // every routing warp's slots are in s_idx / s_w
+      if (warp == 3) {
+        const int TK = T * K;
+        for (int e = lane; e < n; e += 32) s_cnt[e] = 0;
+        __syncwarp();
+        // rank of slot i within its expert, in slot order (t, then k): 32
+        // slots at a time, equal experts in one batch ranked by lane
+        for (int i0 = 0; i0 < TK; i0 += 32) {
+          const int i = i0 + lane;
+          const bool act = i < TK;
+          const int e = act ? s_idx[i] : -1 - lane;
+          const unsigned peers = __match_any_sync(0xffffffffu, e);
+          const int before = __popc(peers & ((1u << lane) - 1u));
+          const int base = act ? s_cnt[e] : 0;
+          __syncwarp();
+          if (act) {
+            s_rank[i] = base + before;
+            if (before == 0) s_cnt[e] = base + __popc(peers);
+          }
+          __syncwarp();
+        }
+        // offsets and the active list: lane l takes experts 8l .. 8l+7
+        int c[8], sum = 0, nact = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int e = lane * 8 + q;
+          c[q] = e < n ? s_cnt[e] : 0;
+          sum += c[q];
+          nact += c[q] > 0 ? 1 : 0;
+        }
+        int incl = sum, inca = nact;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          const int ya = __shfl_up_sync(0xffffffffu, inca, o);
+          if (lane >= o) {
+            incl += y;
+            inca += ya;
+          }
+        }
+        int run = incl - sum, pos = inca - nact;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int e = lane * 8 + q;
+          if (e < n) {
+            s_off[e] = run;
+            run += c[q];
+            if (c[q] > 0) s_active[pos++] = e;
+          }
+        }
+        if (lane == 31) {
+          s_off[n] = incl;
+          s_total = S + inca * nc;
+        }
+        __syncwarp();
+        for (int i = lane; i < TK; i += 32) s_tok[s_off[s_idx[i]] + s_rank[i]] = i / K;
+        __syncwarp();
+        mbar_arrive(tables_bar);  // release: every lane's table writes
+      }
+    }
+  }
+  if (warp >= 4) {
     // ----------------------------------------------------------- epilogue ----
     const int q4 = warp - 4;            // TMEM lane quarter
     const int r = q4 * 32 + lane;       // TMEM lane: W13 block row / W2 row in a tile
@@ -526,7 +640,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
       if (++q == kDecQueue) { q = 0; qphase ^= 1u; }
       if (ud.kind < 0) break;  // the same descriptor in every warp
       // D1 -> SwiGLU -> a^T (bf16, the B operand of the down MMAs)
-      if (!epi_all(warp_wait(gu_full, j & 1u, abort_p, a.status))) break;
+      if (!epi_all(warp_wait(gu_full(j), (j >> 1) & 1u, abort_p, a.status))) break;
       tc_fence_after();
       float z[kDecN];
       tmem_ld16(tl + (j & 1u) * kDecN, z);
@@ -587,50 +701,68 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // one warp per (token, 4 columns): the lanes share the token's partial
-  // rows (shared units with gate 1, then each routed slot's chunks with its
-  // gate), each lane in a fixed order, then a fixed shuffle tree
-  const int cols4 = D / 4;
+  // one CTA per (token, 256 columns): warp w sums the token's partial rows
+  // w, w + 8, ... (shared units with gate 1, then each routed slot's chunks
+  // with its gate) in that order, lane l over columns 8l .. 8l + 7, 8 rows'
+  // loads in flight; then thread c adds the 8 warps' sums of column c in
+  // warp order, adds u and rounds once.  The warps' sums go to the ring,
+  // which the units no longer use.
+  constexpr int kRows = 8;
   const int R = S + K * nc;
-  const int gwarps = static_cast<int>(gridDim.x) * (kDecThreads / 32);
-  for (int item = static_cast<int>(blockIdx.x) * (kDecThreads / 32) + warp; item < T * cols4;
-       item += gwarps) {
-    const int t = item / cols4;
-    const int col = (item - t * cols4) * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int jr = lane; jr < R; jr += 32) {
-      int64_t row;
-      float g;
-      if (jr < S) {
-        row = static_cast<int64_t>(jr) * T + t;
-        g = 1.0f;
-      } else {
-        const int kk = (jr - S) / nc, c = (jr - S) - kk * nc;
-        const int e = s_idx[t * K + kk];
-        row = static_cast<int64_t>(S) * T + static_cast<int64_t>(s_off[e]) * nc +
-              static_cast<int64_t>(c) * s_cnt[e] + s_rank[t * K + kk];
-        g = __ldcg(a.w + t * K + kk);
-      }
-      const float4 p = __ldcg(reinterpret_cast<const float4*>(a.part + row * D + col));
-      acc.x = fmaf(g, p.x, acc.x); acc.y = fmaf(g, p.y, acc.y);
-      acc.z = fmaf(g, p.z, acc.z); acc.w = fmaf(g, p.w, acc.w);
-    }
+  float* wsum = reinterpret_cast<float*>(ring);  // [8 warps][256 columns]
+  for (int item = blockIdx.x; item < T * NV; item += gridDim.x) {
+    const int t = item / NV;
+    const int col0 = (item - t * NV) * 256;
+    const int col = col0 + lane * 8;
+    float acc[8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
-      acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
-      acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
-      acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+    for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+    for (int j0 = warp; j0 < R; j0 += 8 * kRows) {
+      float4 p0[kRows], p1[kRows];
+      float g[kRows];
+#pragma unroll
+      for (int q = 0; q < kRows; ++q) {
+        const int jr = j0 + 8 * q;
+        g[q] = 0.0f;
+        if (jr < R) {
+          int64_t row;
+          if (jr < S) {
+            row = static_cast<int64_t>(jr) * T + t;
+            g[q] = 1.0f;
+          } else {
+            const int kk = (jr - S) / nc, c = (jr - S) - kk * nc;
+            const int e = s_idx[t * K + kk];
+            row = static_cast<int64_t>(S) * T + static_cast<int64_t>(s_off[e]) * nc +
+                  static_cast<int64_t>(c) * s_cnt[e] + s_rank[t * K + kk];
+            g[q] = s_w[t * K + kk];
+          }
+          const float4* src = reinterpret_cast<const float4*>(a.part + row * D + col);
+          p0[q] = __ldcg(src);
+          p1[q] = __ldcg(src + 1);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < kRows; ++q) {
+        if (j0 + 8 * q < R) {
+          acc[0] = fmaf(g[q], p0[q].x, acc[0]); acc[1] = fmaf(g[q], p0[q].y, acc[1]);
+          acc[2] = fmaf(g[q], p0[q].z, acc[2]); acc[3] = fmaf(g[q], p0[q].w, acc[3]);
+          acc[4] = fmaf(g[q], p1[q].x, acc[4]); acc[5] = fmaf(g[q], p1[q].y, acc[5]);
+          acc[6] = fmaf(g[q], p1[q].z, acc[6]); acc[7] = fmaf(g[q], p1[q].w, acc[7]);
+        }
+      }
     }
-    if (lane == 0) {
-      const uint2 uv = *reinterpret_cast<const uint2*>(a.u + static_cast<int64_t>(t) * D + col);
-      __nv_bfloat162 lo = __floats2bfloat162_rn(bf_lo(uv.x) + acc.x, bf_hi(uv.x) + acc.y);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(bf_lo(uv.y) + acc.z, bf_hi(uv.y) + acc.w);
-      uint2 o;
-      o.x = *reinterpret_cast<uint32_t*>(&lo);
-      o.y = *reinterpret_cast<uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(a.h + static_cast<int64_t>(t) * D + col) = o;
+    float4* dst = reinterpret_cast<float4*>(wsum + warp * 256 + lane * 8);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    __syncthreads();
+    {
+      float v = wsum[tid];
+#pragma unroll
+      for (int w8 = 1; w8 < kDecThreads / 32; ++w8) v += wsum[w8 * 256 + tid];
+      const int64_t o = static_cast<int64_t>(t) * D + col0 + tid;
+      a.h[o] = __float2bfloat16_rn(__bfloat162float(a.u[o]) + v);
     }
+    __syncthreads();  // wsum is rewritten by the next item
   }
 }
 
