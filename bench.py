@@ -53,11 +53,14 @@ PER_CONFIG = ("small", "16b", "decode1", "decode8", "decode32", "decode128")
 
 
 def load_peaks():
+    """The roofline denominators: MEASURED_PEAKS.json where present (any key
+    it lacks from the fallback figures), else the fallback figures."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return d, "measured"
-    return FALLBACK_PEAKS, "fallback"
+        peaks = {k: float(d.get(k, v)) for k, v in FALLBACK_PEAKS.items()}
+        return peaks, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json)"
 
 
 def workload_desc(wl):
@@ -241,25 +244,34 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------- our arm
-def kernel_source_hash():
+# the source files each roofline kernel is built from: a traffic record counts
+# only while they are unchanged
+KERNEL_SOURCES = {
+    "gate_up": ("gemm_sm100", "sm100_ptx", "common.cuh"),
+    "decode_layer": ("decode_fused", "sm100_ptx", "common.cuh"),
+}
+
+
+def kernel_source_hash(kind="gate_up"):
     p = os.path.join(ROOT, "mixture_experts_layer_56_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(p)):
-        if f.startswith("gemm_sm100") or f.startswith("sm100_ptx"):
+        if f.startswith(KERNEL_SOURCES[kind]):
             h.update(open(os.path.join(p, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(config_name):
-    """DRAM bytes per launch of the gate/up GEMM from a committed ncu summary,
-    if it was taken on the current kernel source and this workload."""
-    p = os.path.join(ROOT, "profiles", "gemm_gate_up_traffic.json")
+def ncu_traffic(config_name, kind="gate_up"):
+    """DRAM bytes per launch of the roofline kernel (`kind`) from the committed
+    ncu record, if it was taken on this workload and the current source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     try:
-        d = json.load(open(p))
-        if d.get("source_hash") == kernel_source_hash() and d.get("workload") == config_name:
-            return d.get("dram_bytes_per_launch")
+        for d in json.load(open(p))["records"]:
+            if (d.get("kind") == kind and d.get("workload") == config_name
+                    and d.get("source_hash") == kernel_source_hash(kind)):
+                return d.get("dram_bytes_per_launch")
     except Exception:
         return None
     return None
@@ -428,8 +440,8 @@ class Bench:
                 "frac_of_burst": achieved / float(self.peaks["bf16_tflops"]),
                 "frac_of_sustained": achieved / float(self.peaks["bf16_tflops_sustained"]),
                 "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS,
-                "peak_source": f"{self.peak_src} bf16 {'sustained' if capped else 'burst'} "
-                               f"(MEASURED_PEAKS.json); datasheet dense bf16 "
+                "peak_source": f"{self.peak_src} bf16 {'sustained' if capped else 'burst'}; "
+                               f"datasheet dense bf16 "
                                f"{DATASHEET_BF16_TFLOPS:.0f} TFLOP/s for frac_of_datasheet",
                 "flops_per_launch": gate_up_flops, "ms_per_launch": gu_ms}
             down_ms = stage_ms.get("grouped_gemm_down")
@@ -453,11 +465,13 @@ class Bench:
             hbm = float(self.peaks["hbm_gbs"])
             achieved = (layer_bytes + act_bytes) / (ms / 1e3) / 1e9
             out["experts_hit"] = int((counts > 0).sum()) + wl.n_shared
+            one_kernel = r["per_forward"] == 1  # the decode layer kernel
             out["roofline"] = {
                 "bound": "hbm", "kernel": "whole layer forward (all kernels of one step)",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "frac_of_datasheet": achieved / DATASHEET_HBM_GBS, "traffic": None,
-                "peak_source": f"{self.peak_src} HBM copy (MEASURED_PEAKS.json)",
+                "frac_of_datasheet": achieved / DATASHEET_HBM_GBS,
+                "traffic": ncu_traffic(wl.name, "decode_layer") if one_kernel else None,
+                "peak_source": f"{self.peak_src} HBM copy",
                 "bytes_per_step": layer_bytes + act_bytes, "ms_per_step": ms,
                 "bytes": "W1/W3/W2 of the hit routed + shared experts, E, u in, h out"}
             name = "grouped_gemm_gate_up_swiglu" if bf16 else "ffn_f32"
