@@ -34,6 +34,10 @@ CASES = [
     # every width a multiple of 512: CTA pairs take 256 x 512 tiles
     W("wide_tiles", T=1100, d=512, n_routed=12, n_shared=2, inter=256, top_k=3),
     W("wide_ragged", T=333, d=1024, n_routed=5, n_shared=1, inter=512, top_k=2, bias_var=0.5),
+    # widths 512 j + 256 (d = 768, 1280): CTA pairs take 256-column tiles; in
+    # pair_mixed the shared gate/up group alone is a multiple of 512 wide
+    W("pair_odd256", T=700, d=768, n_routed=6, n_shared=1, inter=384, top_k=2),
+    W("pair_mixed", T=600, d=1280, n_routed=10, n_shared=2, inter=640, top_k=3, bias_var=0.5),
 ]
 
 
@@ -53,11 +57,12 @@ def test_bf16_cases_full(wl, mode):
     print(wl.name, mode, {k: v for k, v in rep.items() if k != "gpu"})
 
 
+@pytest.mark.parametrize("d,inter", [(512, 256), (768, 384)], ids=["w512", "w768"])
 @pytest.mark.parametrize("mode", sorted(GEMM_MODES))
-def test_gemm_tile_modes_agree(mode):
+def test_gemm_tile_modes_agree(mode, d, inter):
     """Both tile shapes give results within the bf16 bar of each other and
     the same routing (the routing does not depend on the GEMM)."""
-    wl = W("modes", T=900, d=512, n_routed=8, n_shared=1, inter=256, top_k=2)
+    wl = W("modes", T=900, d=d, n_routed=8, n_shared=1, inter=inter, top_k=2)
     x = S.make_inputs(wl)
     a = P.gpu_stages(x, flags=GEMM_MODES[mode])
     b = P.gpu_stages(x, flags=0)
