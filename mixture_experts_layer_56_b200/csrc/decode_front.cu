@@ -6,14 +6,18 @@
 // the logits are 2 T d N_r FLOPs, the dispatch a few hundred slots.  Here
 // they run on one CTA per token with a single grid-wide step:
 //  A/B. CTA c routes token c (and c + G, ...): the token's row in registers,
-//     warp w forms u_t . e_i for experts w, w + 8, ... as one fp32 FMA chain
-//     per lane plus a fixed shuffle tree, into shared memory; warp 0 then
-//     runs softmax and top-K (lower expert index first on ties, gates not
-//     renormalised) and writes idx / w;
-//  C. after every token is routed: each CTA builds the stable counting sort
-//     of the T*K slots (warp ballots per 32 tokens, as the one-block
-//     dispatch does), CTA 0 writes counts / offsets / perm / inv, and CTA c
-//     copies its tokens' rows of u to their K positions of X_perm.
+//     warp w forms u_t . e_i for experts w, w + 8, ... (four rows in flight)
+//     as one fp32 FMA chain per lane plus a fixed shuffle tree, into shared
+//     memory; then thread i takes expert i: softmax over the block
+//     (fixed-order max and sum) and its rank among the keys (larger first,
+//     lower expert index first on ties) is its slot if below K; gates are
+//     not renormalised;
+//  C. after every token is routed, each CTA sorts the T*K slots by expert,
+//     stably (a counting sort: warp w ranks the slots of its contiguous
+//     range within their experts, 32 at a time by warp match / popc; a block
+//     scan gives the experts' offsets and each range's start within them),
+//     CTA 0 writes counts / offsets / perm / inv, and CTA c copies its
+//     tokens' rows of u to their K positions of X_perm.
 // The grid is at most one CTA per SM, so all of it is resident; the grid-wide
 // step is a counter in the workspace (zeroed before the launch) with a
 // bounded wait.  Results equal moe_route + moe_dispatch + the gather up to
@@ -69,7 +73,7 @@ __device__ __forceinline__ bool grid_step(int* counter, int n, int32_t* status) 
   return ok != 0;
 }
 
-template <int NV, int NW>
+template <int NV>
 __global__ void __launch_bounds__(kFrThreads, 1)
 decode_front_kernel(const bf16* __restrict__ u, const bf16* __restrict__ E,
                     const float* __restrict__ bias, int T, int n, int K, int flags,
@@ -78,16 +82,18 @@ decode_front_kernel(const bf16* __restrict__ u, const bf16* __restrict__ E,
                     int32_t* __restrict__ perm, int32_t* __restrict__ inv, bf16* __restrict__ xperm,
                     FrontSync* sync, int32_t* status) {
   constexpr int D = NV * 256;
-  __shared__ int wc[4][256];
-  __shared__ int tot[256];
-  __shared__ int spos[kDispatchChunk][32];
+  __shared__ int s_slot_e[kDispatchChunk * 32];  // expert of slot t*K + k
+  __shared__ int s_pos[kDispatchChunk * 32];     // rank within (range, expert), then position
+  __shared__ int s_wcnt[kFrWarps][256];          // per warp range and expert: slots, then start
+  __shared__ int s_wsum[kFrWarps];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = static_cast<int>(gridDim.x);
   pdl_wait();
   pdl_trigger();
 
   // ---- A. logits and B. softmax / top-K, one CTA per token ------------------
-  __shared__ float s_logit[256];
+  __shared__ float s_logit[256], s_key[256];
+  __shared__ float s_red[2][kFrWarps];
   const bool select_only = (flags & MOE_FLAG_BIAS_SELECT_ONLY) != 0;
   for (int t = blockIdx.x; t < T; t += G) {
     // the token's row stays in registers; warp w takes experts w, w + 8, ...,
@@ -96,98 +102,82 @@ decode_front_kernel(const bf16* __restrict__ u, const bf16* __restrict__ E,
     uint4 uv[NV];
 #pragma unroll
     for (int v = 0; v < NV; ++v) uv[v] = ur[v * 32 + lane];
-    for (int e0 = warp; e0 < n; e0 += 2 * kFrWarps) {
-      const int e1 = e0 + kFrWarps;
-      const uint4* er0 = reinterpret_cast<const uint4*>(E + static_cast<int64_t>(e0) * D);
-      const uint4* er1 = reinterpret_cast<const uint4*>(E + static_cast<int64_t>(e1 < n ? e1 : e0) * D);
-      uint4 x0[NV], x1[NV];
+    for (int e0 = warp; e0 < n; e0 += 4 * kFrWarps) {
+      uint4 x[4][NV];
 #pragma unroll
-      for (int v = 0; v < NV; ++v) {
-        x0[v] = er0[v * 32 + lane];
-        x1[v] = er1[v * 32 + lane];
+      for (int j = 0; j < 4; ++j) {
+        const int e = e0 + j * kFrWarps;
+        const uint4* er = reinterpret_cast<const uint4*>(E + static_cast<int64_t>(e < n ? e : e0) * D);
+#pragma unroll
+        for (int v = 0; v < NV; ++v) x[j][v] = er[v * 32 + lane];
       }
-      float a0 = 0.0f, a1 = 0.0f;
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
         const float u0 = bf_lo(uv[v].x), u1 = bf_hi(uv[v].x), u2 = bf_lo(uv[v].y),
                     u3 = bf_hi(uv[v].y), u4 = bf_lo(uv[v].z), u5 = bf_hi(uv[v].z),
                     u6 = bf_lo(uv[v].w), u7 = bf_hi(uv[v].w);
-        a0 = fmaf(u0, bf_lo(x0[v].x), a0); a0 = fmaf(u1, bf_hi(x0[v].x), a0);
-        a0 = fmaf(u2, bf_lo(x0[v].y), a0); a0 = fmaf(u3, bf_hi(x0[v].y), a0);
-        a0 = fmaf(u4, bf_lo(x0[v].z), a0); a0 = fmaf(u5, bf_hi(x0[v].z), a0);
-        a0 = fmaf(u6, bf_lo(x0[v].w), a0); a0 = fmaf(u7, bf_hi(x0[v].w), a0);
-        a1 = fmaf(u0, bf_lo(x1[v].x), a1); a1 = fmaf(u1, bf_hi(x1[v].x), a1);
-        a1 = fmaf(u2, bf_lo(x1[v].y), a1); a1 = fmaf(u3, bf_hi(x1[v].y), a1);
-        a1 = fmaf(u4, bf_lo(x1[v].z), a1); a1 = fmaf(u5, bf_hi(x1[v].z), a1);
-        a1 = fmaf(u6, bf_lo(x1[v].w), a1); a1 = fmaf(u7, bf_hi(x1[v].w), a1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 y = x[j][v];
+          float a = acc[j];
+          a = fmaf(u0, bf_lo(y.x), a); a = fmaf(u1, bf_hi(y.x), a);
+          a = fmaf(u2, bf_lo(y.y), a); a = fmaf(u3, bf_hi(y.y), a);
+          a = fmaf(u4, bf_lo(y.z), a); a = fmaf(u5, bf_hi(y.z), a);
+          a = fmaf(u6, bf_lo(y.w), a); a = fmaf(u7, bf_hi(y.w), a);
+          acc[j] = a;
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
-        a0 += __shfl_xor_sync(kFull, a0, o);
-        a1 += __shfl_xor_sync(kFull, a1, o);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] += __shfl_xor_sync(kFull, acc[j], o);
       }
       if (lane == 0) {
-        s_logit[e0] = a0;
-        if (e1 < n) s_logit[e1] = a1;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (e0 + j * kFrWarps < n) s_logit[e0 + j * kFrWarps] = acc[j];
       }
     }
     __syncthreads();
-    if (warp == 0) {
-      float lg[8], key[8], ex[8];
-      float m = -CUDART_INF_F;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int e = lane + 32 * q;
-        float l = -CUDART_INF_F, kv = -CUDART_INF_F;
-        if (e < n) {
-          const float raw = s_logit[e];
-          kv = raw + (bias ? bias[e] : 0.0f);
-          l = select_only ? raw : kv;
-        }
-        lg[q] = l;
-        key[q] = kv;
-        m = fmaxf(m, l);
+    // thread e takes expert e (n <= kFrThreads)
+    {
+      const int e = tid;
+      float l = -CUDART_INF_F, key = -CUDART_INF_F;
+      if (e < n) {
+        const float raw = s_logit[e];
+        key = raw + (bias ? bias[e] : 0.0f);
+        l = select_only ? raw : key;
+        s_key[e] = key;
       }
+      float m = l;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-      float z = 0.0f;
+      if (lane == 0) s_red[0][warp] = m;
+      __syncthreads();
+      m = s_red[0][0];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        ex[q] = (lane + 32 * q < n) ? expf(lg[q] - m) : 0.0f;
-        z += ex[q];
-      }
+      for (int w8 = 1; w8 < kFrWarps; ++w8) m = fmaxf(m, s_red[0][w8]);
+      const float ex = e < n ? expf(l - m) : 0.0f;
+      float z = ex;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
-      const float inv_z = 1.0f / z;
-      unsigned taken = 0;
-      for (int k = 0; k < K; ++k) {
-        float bv = -CUDART_INF_F;
-        int bi = 0x7fffffff;
+      if (lane == 0) s_red[1][warp] = z;
+      __syncthreads();
+      z = s_red[1][0];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int e = lane + 32 * q;
-          if (!((taken >> q) & 1u) && e < n && (key[q] > bv || bi == 0x7fffffff)) {
-            bv = key[q];
-            bi = e;
-          }
+      for (int w8 = 1; w8 < kFrWarps; ++w8) z += s_red[1][w8];
+      if (e < n) {
+        // rank: keys above this one, or equal to it at a lower index
+        int rank = 0;
+#pragma unroll 4
+        for (int j = 0; j < n; ++j) {
+          const float kj = s_key[j];
+          rank += static_cast<int>(kj > key) | (static_cast<int>(kj == key) & static_cast<int>(j < e));
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(kFull, bv, o);
-          const int oi = __shfl_xor_sync(kFull, bi, o);
-          if (ov > bv || (ov == bv && oi < bi)) {
-            bv = ov;
-            bi = oi;
-          }
-        }
-        if ((bi & 31) == lane) {
-          taken |= 1u << (bi >> 5);
-          float g = 0.0f;
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (q == (bi >> 5)) g = ex[q];
-          idx[t * K + k] = bi;
-          w[t * K + k] = g * inv_z;
+        if (rank < K) {
+          idx[t * K + rank] = e;
+          w[t * K + rank] = ex * (1.0f / z);
         }
       }
     }
@@ -196,101 +186,69 @@ decode_front_kernel(const bf16* __restrict__ u, const bf16* __restrict__ E,
   if (!grid_step(&sync->select_done, G, status)) return;
 
   // ---- C. dispatch and gather -------------------------------------------------
-  // warps 0-3: one token per thread (T <= 128), the experts it chose as bits
-  for (int i = tid; i < 4 * 256; i += kFrThreads) (&wc[0][0])[i] = 0;
-  int ek[32];
-  uint32_t mask[NW];
-#pragma unroll
-  for (int v = 0; v < NW; ++v) mask[v] = 0;
-  const bool ranker = warp < 4;  // warp-uniform
-  const int t = tid;
-  if (ranker) {
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      ek[k] = (t < T && k < K) ? __ldcg(idx + t * K + k) : -1;
-#pragma unroll
-      for (int v = 0; v < NW; ++v)
-        if (ek[k] >= 0 && (ek[k] >> 5) == v) mask[v] |= 1u << (ek[k] & 31);
+  const int TK = T * K;
+  for (int i = tid; i < kFrWarps * 256; i += kFrThreads) (&s_wcnt[0][0])[i] = 0;
+  for (int i = tid; i < TK; i += kFrThreads) s_slot_e[i] = __ldcg(idx + i);
+  __syncthreads();
+  // 1. warp w ranks the slots of its range [w per, (w + 1) per) within their
+  //    experts, in slot order: 32 at a time, equal experts ranked by lane
+  const int per = (TK + kFrWarps - 1) / kFrWarps;
+  const int i_lo = min(warp * per, TK), i_hi = min(i_lo + per, TK);
+  for (int i0 = i_lo; i0 < i_hi; i0 += 32) {
+    const int i = i0 + lane;
+    const bool act = i < i_hi;
+    const int e = act ? s_slot_e[i] : -1 - lane;
+    const unsigned peers = __match_any_sync(kFull, e);
+    const int before = __popc(peers & ((1u << lane) - 1u));
+    const int base = act ? s_wcnt[warp][e] : 0;
+    __syncwarp();
+    if (act) {
+      s_pos[i] = base + before;
+      if (before == 0) s_wcnt[warp][e] = base + __popc(peers);
     }
-  }
-  __syncthreads();  // wc is zero
-  if (ranker) {
-#pragma unroll
-    for (int v = 0; v < NW; ++v) {
-      const uint32_t um = __reduce_or_sync(kFull, mask[v]);
-      for (uint32_t m = um; m != 0; m &= m - 1) {
-        const int b = __ffs(m) - 1;
-        const unsigned bal = __ballot_sync(kFull, (mask[v] >> b) & 1u);
-        if (lane == 0) wc[warp][v * 32 + b] = __popc(bal);
-      }
-    }
+    __syncwarp();
   }
   __syncthreads();
-  for (int e = tid; e < 256; e += kFrThreads) {
+  // 2. thread e: the expert's count, its offset (block exclusive scan in
+  //    expert order) and each warp range's start within the expert
+  {
+    const int e = tid;  // kFrThreads == 256 >= n
     int c = 0;
     if (e < n)
-      for (int v = 0; v < 4; ++v) c += wc[v][e];
-    tot[e] = c;
-    if (blockIdx.x == 0 && e < n) counts[e] = c;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    // exclusive scan over the experts, eight entries a lane
-    int v8[8], sum = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v8[i] = tot[lane * 8 + i];
-      sum += v8[i];
-    }
-    int incl = sum;
+      for (int w8 = 0; w8 < kFrWarps; ++w8) c += s_wcnt[w8][e];
+    int incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(kFull, incl, o);
       if (lane >= o) incl += y;
     }
-    int run = incl - sum;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane * 8 + i;
-      tot[e] = run;
-      if (blockIdx.x == 0 && e < n) offsets[e] = run;
-      run += v8[i];
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w8 = 0; w8 < warp; ++w8) before += s_wsum[w8];
+    const int off = before + incl - c;
+    if (blockIdx.x == 0 && e < n) {
+      counts[e] = c;
+      offsets[e] = off;
+      if (e == n - 1) offsets[n] = off + c;
     }
-    if (blockIdx.x == 0 && lane == 31) offsets[n] = incl;
-  }
-  __syncthreads();
-  for (int e = tid; e < n; e += kFrThreads) {
-    int run = tot[e];
-    for (int v = 0; v < 4; ++v) {
-      const int c = wc[v][e];
-      wc[v][e] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
-  if (ranker) {
-    const unsigned lt = (1u << lane) - 1u;
-#pragma unroll
-    for (int v = 0; v < NW; ++v) {
-      const uint32_t um = __reduce_or_sync(kFull, mask[v]);
-      for (uint32_t m = um; m != 0; m &= m - 1) {
-        const int b = __ffs(m) - 1;
-        const int e = v * 32 + b;
-        const bool has = (mask[v] >> b) & 1u;
-        const unsigned bal = __ballot_sync(kFull, has);
-        if (has) {
-          const int pos = wc[warp][e] + __popc(bal & lt);
-          int kk = 0;
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (ek[k] == e) kk = k;
-          if (blockIdx.x == 0) {
-            perm[pos] = t * K + kk;
-            inv[t * K + kk] = pos;
-          }
-          spos[t][kk] = pos;
-        }
+    if (e < n) {
+      int run = off;
+      for (int w8 = 0; w8 < kFrWarps; ++w8) {
+        const int cw = s_wcnt[w8][e];
+        s_wcnt[w8][e] = run;
+        run += cw;
       }
+    }
+  }
+  __syncthreads();
+  // 3. each slot's position: its range's start within the expert + its rank
+  for (int i = tid; i < TK; i += kFrThreads) {
+    const int pos = s_wcnt[i / per][s_slot_e[i]] + s_pos[i];
+    s_pos[i] = pos;
+    if (blockIdx.x == 0) {
+      perm[pos] = i;
+      inv[i] = pos;
     }
   }
   __syncthreads();
@@ -302,7 +260,7 @@ decode_front_kernel(const bf16* __restrict__ u, const bf16* __restrict__ E,
 #pragma unroll
     for (int j = 0; j < NV; ++j) v[j] = src[j * 32 + lane];
     for (int kk = warp; kk < K; kk += kFrWarps) {
-      uint4* dst = reinterpret_cast<uint4*>(xperm + static_cast<int64_t>(spos[tt][kk]) * D);
+      uint4* dst = reinterpret_cast<uint4*>(xperm + static_cast<int64_t>(s_pos[tt * K + kk]) * D);
 #pragma unroll
       for (int j = 0; j < NV; ++j) dst[j * 32 + lane] = v[j];
     }
@@ -314,19 +272,10 @@ int launch_front_nv(const moe_shape_t& s, const void* u, const void* E, const fl
                     int32_t* idx, float* w, float* logits, int32_t* counts, int32_t* offsets,
                     int32_t* perm, int32_t* inv, void* xperm, FrontSync* sync, int32_t* status,
                     int grid, cudaStream_t st) {
-  const int nw = (s.n_routed + 31) / 32;
-#define MOE_FRONT_CASE(W)                                                                      \
-  case W:                                                                                      \
-    return launch_k(decode_front_kernel<NV, W>, grid, kFrThreads, 0, st, 1,                    \
-                    static_cast<const bf16*>(u), static_cast<const bf16*>(E), bias,            \
-                    static_cast<int>(s.T), s.n_routed, s.top_k, s.flags, idx, w, logits, counts, \
-                    offsets, perm, inv, static_cast<bf16*>(xperm), sync, status);
-  switch (nw) {
-    MOE_FRONT_CASE(1) MOE_FRONT_CASE(2) MOE_FRONT_CASE(3) MOE_FRONT_CASE(4)
-    MOE_FRONT_CASE(5) MOE_FRONT_CASE(6) MOE_FRONT_CASE(7) MOE_FRONT_CASE(8)
-    default: return MOE_ERR_SHAPE;
-  }
-#undef MOE_FRONT_CASE
+  return launch_k(decode_front_kernel<NV>, grid, kFrThreads, 0, st, 1,
+                  static_cast<const bf16*>(u), static_cast<const bf16*>(E), bias,
+                  static_cast<int>(s.T), s.n_routed, s.top_k, s.flags, idx, w, logits, counts,
+                  offsets, perm, inv, static_cast<bf16*>(xperm), sync, status);
 }
 
 }  // namespace
