@@ -36,14 +36,24 @@ constexpr int BK = 64;
 constexpr int kThreads = 384;  // 4 role warps + 8 epilogue warps
 constexpr int kMaxGroups = 257;  // 256 routed + 1 shared
 
-template <int BN> struct Cfg;
-template <> struct Cfg<256> { static constexpr int STAGES = 4; };
-template <> struct Cfg<128> { static constexpr int STAGES = 6; };
-template <> struct Cfg<64>  { static constexpr int STAGES = 8; };
+// Stage layout by the N tile BN and the A rows a stage holds, AR: 128, or 64
+// / 32 for batches whose groups have at most that many rows (fewer than 128
+// tokens).  The MMA still reads 128 rows of A from the stage's start; the
+// rows past AR are other bytes of the same stage (AR * 128 + BN * 128 >=
+// 16 KB), their accumulator rows never stored.  Smaller A leaves room for
+// more stages of B, the weights that decode-sized batches stream.
+template <int BN, int AR> struct Cfg {
+  static constexpr int kBytes = AR * BK * 2 + BN * BK * 2;
+  static constexpr int STAGES = (216 * 1024) / kBytes < 32 ? (216 * 1024) / kBytes : 32;
+  static_assert(kBytes >= BM * BK * 2, "the MMA's 128 rows of A stay inside the stage");
+};
+template <> struct Cfg<256, 128> { static constexpr int STAGES = 4; };
+template <> struct Cfg<128, 128> { static constexpr int STAGES = 6; };
+template <> struct Cfg<64, 128>  { static constexpr int STAGES = 8; };
 
-template <int BN>
+template <int BN, int AR>
 constexpr int smem_bytes() {
-  return Cfg<BN>::STAGES * (BM * BK * 2 + BN * BK * 2) + 1024;
+  return Cfg<BN, AR>::STAGES * (AR * BK * 2 + BN * BK * 2) + 1024;
 }
 
 struct TileInfo {
@@ -70,13 +80,13 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int32_t* tile_st
   return t;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int AR>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
                     const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
                     const GroupedGemmArgs args) {
-  constexpr int STAGES = Cfg<BN>::STAGES;
-  constexpr uint32_t A_BYTES = BM * BK * 2;
+  constexpr int STAGES = Cfg<BN, AR>::STAGES;
+  constexpr uint32_t A_BYTES = AR * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -183,7 +193,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
         tma_prefetch_desc(&tmB_s);
       }
       const uint32_t a_bytes =
-          static_cast<uint32_t>(args.a_rows > 0 && args.a_rows < BM ? args.a_rows : BM) * BK * 2;
+          static_cast<uint32_t>(args.a_rows > 0 && args.a_rows < AR ? args.a_rows : AR) * BK * 2;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, issued_parity = 0;
@@ -400,27 +410,38 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, 
   return res == CUDA_SUCCESS;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int AR>
 static int launch_impl(const GemmMaps& m, const GroupedGemmArgs& args, int grid,
                        cudaStream_t stream) {
   static std::atomic<uint64_t> optin{0};
-  auto kern = grouped_gemm_kernel<BN, EPI>;
-  if (int rc = ensure_smem_optin(reinterpret_cast<const void*>(kern), smem_bytes<BN>(), optin))
-    return rc;
-  return launch_k(kern, grid, kThreads, smem_bytes<BN>(), stream, 1, m.a_r, m.a_s, m.b_r, m.b_s,
-                  args);
+  auto kern = grouped_gemm_kernel<BN, EPI, AR>;
+  constexpr int smem = smem_bytes<BN, AR>();
+  if (int rc = ensure_smem_optin(reinterpret_cast<const void*>(kern), smem, optin)) return rc;
+  return launch_k(kern, grid, kThreads, smem, stream, 1, m.a_r, m.a_s, m.b_r, m.b_s, args);
+}
+
+// the stage layout for the A rows of the batch (a_rows 0 means 128)
+template <int BN, int EPI>
+static int launch_rows(const GemmMaps& m, const GroupedGemmArgs& args, int grid,
+                       cudaStream_t stream) {
+  const int ar = args.a_rows > 0 ? args.a_rows : BM;
+  if constexpr (BN >= 128) {
+    if (ar <= 32) return launch_impl<BN, EPI, 32>(m, args, grid, stream);
+  }
+  if (ar <= 64) return launch_impl<BN, EPI, 64>(m, args, grid, stream);
+  return launch_impl<BN, EPI, 128>(m, args, grid, stream);
 }
 
 int launch_grouped_gemm(int BN, int epi, const GemmMaps& maps, const GroupedGemmArgs& args,
                         int grid, cudaStream_t stream) {
   if (grid <= 0) return MOE_OK;
   if (epi == kEpiSwiGLU) {
-    if (BN == 256) return launch_impl<256, kEpiSwiGLU>(maps, args, grid, stream);
-    if (BN == 128) return launch_impl<128, kEpiSwiGLU>(maps, args, grid, stream);
+    if (BN == 256) return launch_rows<256, kEpiSwiGLU>(maps, args, grid, stream);
+    if (BN == 128) return launch_rows<128, kEpiSwiGLU>(maps, args, grid, stream);
   } else {
-    if (BN == 256) return launch_impl<256, kEpiPlain>(maps, args, grid, stream);
-    if (BN == 128) return launch_impl<128, kEpiPlain>(maps, args, grid, stream);
-    if (BN == 64) return launch_impl<64, kEpiPlain>(maps, args, grid, stream);
+    if (BN == 256) return launch_rows<256, kEpiPlain>(maps, args, grid, stream);
+    if (BN == 128) return launch_rows<128, kEpiPlain>(maps, args, grid, stream);
+    if (BN == 64) return launch_rows<64, kEpiPlain>(maps, args, grid, stream);
   }
   return MOE_ERR_SHAPE;
 }
