@@ -247,7 +247,8 @@ def run_reference(args):
 # the source files each roofline kernel is built from: a traffic record counts
 # only while they are unchanged
 KERNEL_SOURCES = {
-    "gate_up": ("gemm_sm100", "sm100_ptx", "common.cuh"),
+    # the prefill layers' gate/up GEMM: the CTA-pair kernels
+    "gate_up": ("gemm_sm100_pair", "gemm_sm100.h", "sm100_ptx", "common.cuh"),
     "decode_layer": ("decode_fused", "sm100_ptx", "common.cuh"),
 }
 
