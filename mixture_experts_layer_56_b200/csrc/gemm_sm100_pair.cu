@@ -731,6 +731,10 @@ grouped_gemm_pair_wide_kernel(const __grid_constant__ CUtensorMap tmA_r,
               Vec16<bf16>::store(reinterpret_cast<bf16*>(&packed[hh * 4 + v]), o);
             }
           }
+          // the half's accumulator is in registers: release it before the stores
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(h ? tempty_leader1 : tempty_leader0);
           uint8_t* dst = live ? reinterpret_cast<uint8_t*>(out + orow * ld + col0) : nullptr;
           warp_store_rows<128>(stage, packed, dst, lane);
         } else if (ti.shared) {
@@ -753,37 +757,37 @@ grouped_gemm_pair_wide_kernel(const __grid_constant__ CUtensorMap tmA_r,
             warp_store_rows<128>(stage, packed, dst, lane);
             if (c + 1 < 4) tmem_ld_wait_regs(x);
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(h ? tempty_leader1 : tempty_leader0);
         } else {
-          // bf16 routed output: 2 chunks of 64 columns (128 bytes a row)
+          // bf16 routed output: 2 chunks of 64 columns (128 bytes a row),
+          // both read from TMEM and packed first, so that the half is
+          // released before the stores
           const int64_t colb = static_cast<int64_t>(ti.n_blk) * kWideBN + h * kWideHalf + hc * 128;
-          float x[64];
-          tmem_ld32(taddr, x);
-          tmem_ld32(taddr + 32, x + 32);
-          tmem_ld_wait_regs(x);
-          tmem_ld_wait_regs(x + 32);
-#pragma unroll 1
+          uint4 packed[2][8];
+#pragma unroll
           for (int c = 0; c < 2; ++c) {
-            uint4 packed[8];
+            float x[64];
+            tmem_ld32(taddr + c * 64, x);
+            tmem_ld32(taddr + c * 64 + 32, x + 32);
+            tmem_ld_wait_regs(x);
+            tmem_ld_wait_regs(x + 32);
 #pragma unroll
             for (int v = 0; v < 8; ++v)
-              Vec16<bf16>::store(reinterpret_cast<bf16*>(&packed[v]), x + v * 8);
-            if (c == 0) {
-              tmem_ld32(taddr + 64, x);
-              tmem_ld32(taddr + 96, x + 32);
-            }
+              Vec16<bf16>::store(reinterpret_cast<bf16*>(&packed[c][v]), x + v * 8);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(h ? tempty_leader1 : tempty_leader0);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
             uint8_t* dst = live ? reinterpret_cast<uint8_t*>(static_cast<bf16*>(args.out_r) +
                                                              prow * args.ld_r + colb + c * 64)
                                 : nullptr;
-            warp_store_rows<128>(stage, packed, dst, lane);
-            if (c == 0) {
-              tmem_ld_wait_regs(x);
-              tmem_ld_wait_regs(x + 32);
-            }
+            warp_store_rows<128>(stage, packed[c], dst, lane);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(h ? tempty_leader1 : tempty_leader0);
       }
     }
   }
