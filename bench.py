@@ -33,6 +33,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -253,12 +254,20 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text):
+    """Source text without its comments and blank lines: a record stays valid
+    across comment edits, not across code changes."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*", "", line).rstrip() for line in text.splitlines())
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_source_hash(kind="gate_up"):
     p = os.path.join(ROOT, "mixture_experts_layer_56_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(p)):
         if f.startswith(KERNEL_SOURCES[kind]):
-            h.update(open(os.path.join(p, f), "rb").read())
+            h.update(_code_only(open(os.path.join(p, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -23,14 +23,15 @@
 //            of them for a shared expert) as partial rows.
 // Roles (8 warps): warp 0 the TMA producer (unit counter, W13 and W2 tiles into
 // an 11-stage ring, running ahead into the next unit), warp 1 the MMA issuer,
-// warp 2 the TMEM owner, warps 4-7 the epilogue (TMEM lane quarters).  The
-// ring carries unit i's W13 tiles before unit i-1's W2 tiles, and D1 is
+// warp 2 the TMEM owner, warps 2-7 the routing of every token and warp 3 the
+// expert tables (phase 2), then warps 4-7 the epilogue (TMEM lane quarters).
+// The ring carries unit i's W13 tiles before unit i-1's W2 tiles, and D1 is
 // double-buffered, so unit i's gate/up MMAs run while the epilogue turns
 // unit i-1's D1 into a^T.
 //
 // Phases, all in this one launch (one CTA per SM):
-//  1. Logits (with G = min(n, grid), CTA c < G takes experts c, c + G, ...): expert
-//     i's row stays in registers while each warp takes two tokens,
+//  1. Logits (with G = min(n, grid), CTA c < G takes experts c, c + G, ...):
+//     expert i's row stays in registers while each warp takes two tokens,
 //     u_t . e_i as fp32 FMA chains per lane plus a fixed shuffle tree; the
 //     CTA publishes its logits and counts itself.
 //  2. Routing and tables (warps 2-7 of every CTA, the same arithmetic in

@@ -62,6 +62,9 @@ def test_traffic_record_follows_its_own_kernel_sources(tmp_path, monkeypatch):
     (csrc / "kernels.cu").write_text("changed")
     (csrc / "gemm_sm100.cu").write_text("changed")          # the single-CTA kernel
     assert bench.ncu_traffic("large") == 10
-    # a change to the CTA-pair kernel's source voids the record
+    # comments and blank lines are not the kernel
+    (csrc / "gemm_sm100_pair.cu").write_text("// a note\ngemm_sm100_pair.cu  /* more */\n\n")
+    assert bench.ncu_traffic("large") == 10
+    # a change to the CTA-pair kernel's code voids the record
     (csrc / "gemm_sm100_pair.cu").write_text("changed")
     assert bench.ncu_traffic("large") is None
