@@ -170,6 +170,24 @@ __device__ __forceinline__ bool spin_until(const int* p, int target, int32_t* st
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
+// Each weight tile is read once per launch: its L2 lines go first, so that
+// the partial rows (written during the units, read back by the combine), the
+// tokens' tiles and the router's inputs stay in L2 while the weights stream.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void tma_load_2d_evict_first(uint32_t dst, const CUtensorMap* map,
+                                                        uint32_t bar, int32_t x, int32_t y,
+                                                        uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
 // Softmax and top-K of tokens t0, t0 + tstep, ... < T, one warp; lane l holds
 // experts l, l + 32, ..., l + 32 (NQ - 1) (NQ * 32 >= n).  keys: this warp's
 // shared row of 4 * ceil(n / 4) floats.  Each selected expert e of token t
@@ -387,6 +405,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer ----
     if (lane == 0) {
+      const uint64_t w_policy = l2_evict_first_policy();
       tma_prefetch_desc(&tmW13);
       tma_prefetch_desc(&tmW2);
       tma_prefetch_desc(&tmU);
@@ -442,7 +461,7 @@ decode_layer_kernel(const __grid_constant__ CUtensorMap tmW13,
           if (!wait_bounded(empty_bar(stage), sphase ^ 1u, abort_p, a.status)) return false;
           const uint32_t dst = ring_base + stage * kDecStageBytes;
           mbar_arrive_expect_tx(full_bar(stage), kDecTileBytes + (with_u ? kDecUTileBytes : 0));
-          tma_load_2d(dst, map, full_bar(stage), x, y);
+          tma_load_2d_evict_first(dst, map, full_bar(stage), x, y, w_policy);
           if (with_u) tma_load_2d(dst + kDecTileBytes, &tmU, full_bar(stage), x, 0);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (sphase << stage);
