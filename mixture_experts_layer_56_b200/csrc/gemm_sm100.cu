@@ -56,6 +56,24 @@ constexpr int smem_bytes() {
   return Cfg<BN, AR>::STAGES * (AR * BK * 2 + BN * BK * 2) + 1024;
 }
 
+// When every group fits one row block (decode-sized batches) each B tile is
+// read by one tile only: its L2 lines go first, so that the rows of A, the
+// outputs and the next kernels' inputs stay in L2 while the weights stream.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void tma_load_3d_evict_first(uint32_t dst, const CUtensorMap* map,
+                                                        uint32_t bar, int32_t x, int32_t y,
+                                                        int32_t z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "l"(policy)
+      : "memory");
+}
+
 struct TileInfo {
   int g;        // group index (0 = shared when present)
   int shared;   // 1 for the shared-expert group
@@ -102,6 +120,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
   __shared__ int32_t tile_start[kMaxGroups + 1];
   __shared__ int32_t grp_row0[kMaxGroups];
   __shared__ int32_t grp_rows[kMaxGroups];
+  __shared__ int b_once;  // every group fits one row block: each B tile is read once
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -169,11 +188,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
       if (lane >= o) incl += v;
     }
     int run = incl - sum;
+    bool big = false;
     for (int i = beg; i < end; ++i) {
       run += tile_start[i + 1];
       tile_start[i + 1] = run;
+      big = big || grp_rows[i] > BM;
     }
-    if (lane == 0) tile_start[0] = 0;
+    big = __any_sync(0xffffffffu, big);
+    if (lane == 0) {
+      tile_start[0] = 0;
+      b_once = big ? 0 : 1;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -194,6 +219,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
       }
       const uint32_t a_bytes =
           static_cast<uint32_t>(args.a_rows > 0 && args.a_rows < AR ? args.a_rows : AR) * BK * 2;
+      const uint64_t b_policy = l2_evict_first_policy();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, issued_parity = 0;
@@ -217,8 +243,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_cons
           const uint32_t sa = smem_base + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(full_bar(stage), a_bytes + B_BYTES);
           tma_load_2d(sa, ma, full_bar(stage), kb * BK, row);
-          tma_load_3d(sa + A_BYTES, mb, full_bar(stage), (kb % args.kb_per_expert) * BK, nrow,
-                      zbase + kb / args.kb_per_expert);
+          if (b_once)
+            tma_load_3d_evict_first(sa + A_BYTES, mb, full_bar(stage),
+                                    (kb % args.kb_per_expert) * BK, nrow,
+                                    zbase + kb / args.kb_per_expert, b_policy);
+          else
+            tma_load_3d(sa + A_BYTES, mb, full_bar(stage), (kb % args.kb_per_expert) * BK, nrow,
+                        zbase + kb / args.kb_per_expert);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
