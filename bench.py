@@ -475,7 +475,8 @@ class Bench:
             hbm = float(self.peaks["hbm_gbs"])
             achieved = (layer_bytes + act_bytes) / (ms / 1e3) / 1e9
             out["experts_hit"] = int((counts > 0).sum()) + wl.n_shared
-            one_kernel = r["per_forward"] == 1  # the decode layer kernel
+            one_kernel = (self.L.moe_forward_path(layer.shape_for(T))
+                          == self.L.MOE_PATH_DECODE_LAYER)  # the decode layer kernel
             out["roofline"] = {
                 "bound": "hbm", "kernel": "whole layer forward (all kernels of one step)",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,

@@ -293,7 +293,9 @@ int launch_decode_front(const moe_shape_t& s, const void* u, const void* E, cons
                         int32_t* perm, int32_t* inv, void* xperm, void* sync, int32_t* status,
                         int sms, cudaStream_t st) {
   const int grid = s.T < sms ? static_cast<int>(s.T) : sms;
-  if (cudaMemsetAsync(sync, 0, sizeof(FrontSync), st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (int rc = launch_zero_words(static_cast<int32_t*>(sync),
+                                 static_cast<int>(sizeof(FrontSync) / sizeof(int32_t)), st))
+    return rc;
   FrontSync* fs = static_cast<FrontSync*>(sync);
   switch (s.d) {
     case 256: return launch_front_nv<1>(s, u, E, bias, idx, w, logits, counts, offsets, perm, inv, xperm, fs, status, grid, st);

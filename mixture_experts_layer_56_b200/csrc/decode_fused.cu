@@ -59,6 +59,7 @@
 #include "common.cuh"
 #include "decode_fused.h"
 #include "gemm_sm100.h"
+#include "kernels.h"
 #include "sm100_ptx.cuh"
 
 namespace moe {
@@ -839,7 +840,9 @@ int launch_decode_fused(const moe_shape_t& s, const void* u, const void* E, cons
   if (!make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u, d, static_cast<uint64_t>(s.T), d * 2,
                    64, kDecN))
     return MOE_ERR_CUDA;
-  if (cudaMemsetAsync(sync, 0, sizeof(DecSync), st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (int rc = launch_zero_words(static_cast<int32_t*>(sync),
+                                 static_cast<int>(sizeof(DecSync) / sizeof(int32_t)), st))
+    return rc;
   DecArgs a{};
   a.u = static_cast<const bf16*>(u);
   a.E = static_cast<const bf16*>(E);

@@ -753,6 +753,16 @@ int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_
   return rc;
 }
 
+__global__ void zero_words_kernel(int32_t* p, int n) {
+  pdl_wait();     // the kernel before may still count on these words
+  pdl_trigger();  // the next kernel's set-up may overlap the writes below
+  for (int i = threadIdx.x; i < n; i += blockDim.x) p[i] = 0;
+}
+
+int launch_zero_words(int32_t* p, int n, cudaStream_t st) {
+  return launch_k(zero_words_kernel, 1, 32, 0, st, 1, p, n);
+}
+
 int launch_gather(int dtype, const void* u, const int32_t* perm, int64_t rows, int d, int K,
                   void* xperm, cudaStream_t st) {
   if (rows == 0) return MOE_OK;

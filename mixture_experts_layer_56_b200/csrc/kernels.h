@@ -44,6 +44,12 @@ int launch_dispatch(const int32_t* idx, int64_t T, int K, int n, int32_t* chunk_
 int launch_gather(int dtype, const void* u, const int32_t* perm, int64_t rows, int d, int K,
                   void* xperm, cudaStream_t st);
 
+// Zeroes the n words at p (the grid-wide counters a decode kernel after it
+// counts on) with a one-warp kernel: it waits for the kernel before it in the
+// stream, which may still use the words, and then lets the next kernel begin
+// its set-up while it writes (programmatic dependent launch).
+int launch_zero_words(int32_t* p, int n, cudaStream_t st);
+
 int launch_combine(int dtype, const void* u, const float* ysh, const void* y, const float* w,
                    const int32_t* inv, int64_t T, int d, int K, void* h, cudaStream_t st);
 

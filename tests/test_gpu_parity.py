@@ -368,7 +368,7 @@ def test_small_batch_front_kernel(wl):
 @pytest.mark.parametrize("T", [4, 64])
 def test_small_paths_replay_from_a_cuda_graph_bitwise(T):
     """The one-kernel decode layer (T = 4) and the small-batch front kernel
-    (T = 64) zero their sync words with a memset node before the kernel:
+    (T = 64) zero their sync words with a one-warp kernel before them:
     captured into a CUDA graph, every replay gives the eager result."""
     wl = W(f"graph{T}", T=T, d=512, n_routed=32, n_shared=1, inter=128, top_k=4)
     x = S.make_inputs(wl)
