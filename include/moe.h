@@ -211,7 +211,8 @@ int moe_combine(const moe_shape_t* shape, const void* u, const float* ysh,
    streams each activated expert's weights once in units of 64 intermediate
    rows, with fp32 partial down projections summed in a fixed order, and
    other batches of up to 128 tokens route, dispatch and gather in one
-   kernel; their h matches the oracle within the same bars but is not the
+   kernel (each after a one-warp kernel that zeroes its grid-wide counters
+   in ws); their h matches the oracle within the same bars but is not the
    stage-wise result bit for bit.  All other batches give exactly the result
    of moe_route, moe_dispatch, moe_expert_ffn and moe_combine. */
 int moe_layer_forward(const moe_shape_t* shape, const void* u, const void* E,
